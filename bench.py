@@ -1,0 +1,455 @@
+"""Benchmark: wave-round attention on the Wan2.1-1.3B-shaped round.
+
+One step = one pass of the whole hot path over one wave round: the round's
+schedule and key tables (host), the K/V append of every active node (one
+kernel each), and the attention of all active nodes in one kernel launch. The
+workload is round 6 of the 7-chunk, 4-level progressive schedule: nodes (2,0)
+[refresh], (3,1), (4,2), (5,3), (6,4); 12 heads, head_dim 128, 4680 tokens per
+chunk; its history K/V (rounds 0..5) is appended once before timing, and each
+step appends the round's own K/V again (released after the step, so every step
+does identical work on identical pages).
+
+Output: one JSON line (rank 0). ``value`` is attention TFLOP/s over the whole
+job (all ranks; algorithmic FLOPs 4*Nq*Nk*d per head, valid tokens only,
+divided by the step time, so append time counts against it). Inputs (K/V cache
+of the round ~0.7 GB, Q 72 MB) exceed the 126 MB L2, so no flush is needed.
+
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only) on a
+bounded sample of the same round.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import wave_inputs as wi  # noqa: E402
+
+METRIC = "wave-round attention TFLOP/s and chunk-updates/s at 1 B200; % of BF16 dense peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "wan2.1-1.3b round 6 (B=7, K=4, progressive)"
+ROUND = 6
+POLICY = "progressive"
+
+
+def _config(extra=None):
+    wl = wi.WAN21
+    cfg = {"workload": WORKLOAD, "heads": wl.heads, "head_dim": wl.head_dim,
+           "tokens_per_chunk": wl.tokens, "chunks": wl.chunks, "levels": wl.levels,
+           "policy": POLICY, "round": ROUND,
+           "active_nodes": "(2,0) refresh, (3,1), (4,2), (5,3), (6,4)",
+           "l2": "inputs larger than L2 (round K/V 0.7 GB, Q 72 MB); no flush"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def _measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(x: float, backend_device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=backend_device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        return self.summary()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+
+class Round:
+    """Host-side description of the timed round, from the library's scheduler."""
+
+    def __init__(self, wave):
+        wl = wi.WAN21
+        self.wl = wl
+        self.rounds = wave.schedule(wl.chunks, wl.levels, POLICY, wl.window)
+        self.last = wave.last_read_rounds(wl.chunks, wl.levels, POLICY, wl.window)
+        self.active = self.rounds[ROUND]
+
+
+def _bits_to_dev(bits, pin=False):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.pin_memory() if pin else t.cuda()
+
+
+def run_gpu(args):
+    import torch
+    import block_causal_attention_wave_b200 as wave
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wave.load()
+    rd = Round(wave)
+    wl = rd.wl
+    page_bytes = wave.KVCache.page_bytes(wl.heads, wl.head_dim)
+    n_pages = 2400  # 1.9 GB: the live cache peaks near 900 pages
+    pool = torch.empty(4096 + n_pages * page_bytes, dtype=torch.uint8, device="cuda")
+    kv = wave.KVCache(wl.heads, wl.head_dim, wl.tokens, wl.levels, wl.window, 0, pool=pool)
+    stream = torch.cuda.current_stream()
+
+    def kvbits(kind, e):
+        return wi.node_tensor(kind, e[0], e[1], wl.tokens, wl.heads, wl.head_dim, wl.scale)
+
+    # Bring the cache to the start of the timed round (untimed).
+    for t in range(ROUND):
+        for n in rd.rounds[t]:
+            kv.append(n[0], n[1], _bits_to_dev(kvbits("k", n)), _bits_to_dev(kvbits("v", n)))
+        for e in sorted(e for e, lr in rd.last.items() if lr == t):
+            kv.release(*e)
+    torch.cuda.synchronize()
+    active = rd.active
+    host_k = [kvbits("k", n) for n in active]
+    host_v = [kvbits("v", n) for n in active]
+    host_q = np.concatenate([kvbits("q", n) for n in active])
+    dk = [_bits_to_dev(b) for b in host_k]
+    dv = [_bits_to_dev(b) for b in host_v]
+    dq = _bits_to_dev(host_q)
+    do = torch.empty_like(dq)
+
+    def append_round():
+        for n, k, v in zip(active, dk, dv):
+            kv.append(n[0], n[1], k, v, stream)
+
+    # FLOPs from the library's own key tables (valid tokens only).
+    append_round()
+    table = kv.gather_table(active, POLICY)
+    for n in active:
+        kv.release(*n)
+    n_keys = [sum(v for _, v in rows) for rows in table]
+    flops = sum(4 * wl.tokens * nk * wl.heads * wl.head_dim for nk in n_keys)
+    upd_nodes = sum(1 for n in active if n[1] > 0)
+    append_bytes = 0
+    for rows in table:
+        pass
+    per_node_read = 2 * wl.tokens * wl.heads * wl.head_dim * 2
+    per_node_write = 2 * math.ceil(wl.tokens / 128) * 128 * wl.heads * wl.head_dim * 2
+    append_bytes = len(active) * (per_node_read + per_node_write)
+
+    def step(ev_a=None, ev_b=None):
+        append_round()
+        if ev_a is not None:
+            ev_a.record(stream)
+        kv.round_attn(active, POLICY, dq, do, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+        for n in active:
+            kv.release(*n)
+
+    for _ in range(args.warmup):
+        step()
+    kv.status(stream)
+
+    # ---- device-timed region
+    K = args.steps
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local)
+    clk.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        step(ev_a[i], ev_b[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = clk.stop()
+    kv.status(stream)
+    ms_local = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    ms = reduce_max(ms_local, "cuda" if ws > 1 else None)
+    ms_step = ms / K
+    value = ws * flops * K / (ms * 1e-3) / 1e12
+    attn_avg = sum(attn_ms) / len(attn_ms)
+
+    # ---- append kernel alone (HBM roofline context)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(5):
+        append_round()
+        for n in active:
+            kv.release(*n)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    append_ms = ea.elapsed_time(eb) / 5 / len(active)
+
+    # ---- end to end through the public API with host buffers
+    hq = _bits_to_dev(host_q, pin=True)
+    hk = [_bits_to_dev(b, pin=True) for b in host_k]
+    hv = [_bits_to_dev(b, pin=True) for b in host_v]
+    ho = torch.empty(dq.shape, dtype=torch.bfloat16, pin_memory=True)
+    h2d = hq.numel() * 2 + sum(x.numel() * 2 for x in hk + hv)
+    d2h = ho.numel() * 2
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        for d, h in zip(dk, hk):
+            d.copy_(h, non_blocking=True)
+        for d, h in zip(dv, hv):
+            d.copy_(h, non_blocking=True)
+        step()
+        ho.copy_(do, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    E = max(3, min(K, 20))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), "cuda" if ws > 1 else None) / E
+    kv.status(stream)
+
+    peaks, src = _measured_peaks()
+    achieved = flops / (attn_avg * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config({"replicas": ws}),
+        "chunk_updates_per_s": round(ws * upd_nodes * K / (ms * 1e-3), 2),
+        "pct_bf16_dense_peak": round(100 * value / ws / peak, 2),
+        "e2e": {"value": round(ws * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "roofline": {"bound": "tensor", "kernel": "round_attn_kernel<128>",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst, cuBLAS 8192^3)",
+                     "flops_per_launch": flops, "avg_launch_ms": round(attn_avg, 4)},
+        "append": {"kernel": "kv_append_kernel", "avg_launch_ms": round(append_ms, 4),
+                   "achieved_gbs": round(append_bytes / len(active) / (append_ms * 1e-3) / 1e9, 1),
+                   "peak_gbs": peaks["hbm_gbs"],
+                   "frac": round(append_bytes / len(active) / (append_ms * 1e-3) / 1e9 /
+                                 peaks["hbm_gbs"], 4)},
+        "gpu_launches": K * (len(active) + 1),
+        "clocks": clocks,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def _oracle_round():
+    """Float64 inputs of the timed round for the oracle (rank 0 only)."""
+    from oracle import cache as ocache
+    from oracle import schedule as osched
+    wl = wi.WAN21
+    active = osched.schedule(wl.chunks, wl.levels, POLICY, wl.window)[ROUND]
+    ents = set()
+    for n in active:
+        ents.update(ocache.key_entries(n, POLICY, wl.window, False))
+
+    def f64(kind, e):
+        return wi.bf16_bits_to_f64(
+            wi.node_tensor(kind, e[0], e[1], wl.tokens, wl.heads, wl.head_dim, wl.scale))
+
+    entries = {e: (f64("k", e), f64("v", e)) for e in sorted(ents)}
+    qs = {n: f64("q", n) for n in active}
+    return active, entries, qs
+
+
+def _sample_rows(n_rows, T):
+    return np.unique(np.linspace(0, T - 1, n_rows).astype(np.int64))
+
+
+def _oracle_sample(active, entries, qs, n_rows):
+    from oracle import attention as oatt
+    wl = wi.WAN21
+    rows = _sample_rows(n_rows, wl.tokens)
+    t = time.perf_counter()
+    oatt.round_attention(active, POLICY, wl.window, qs, entries, None,
+                         {n: rows for n in active})
+    dt = time.perf_counter() - t
+    n_keys = {n: (len(active) and None) for n in active}
+    flops = 0
+    from oracle import cache as ocache
+    for n in active:
+        nk = len(ocache.key_entries(n, POLICY, wl.window, False)) * wl.tokens
+        flops += 4 * len(rows) * nk * wl.heads * wl.head_dim
+    del n_keys
+    return dt, flops, len(rows)
+
+
+def _cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(i.get("num_threads", 1) for i in info) if info else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(target_s=10.0):
+    active, entries, qs = _oracle_round()
+    dt, _, _ = _oracle_sample(active, entries, qs, 16)
+    n_rows = int(min(1024, max(16, 16 * target_s / max(dt, 1e-3))))
+    dt, flops, nr = _oracle_sample(active, entries, qs, n_rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": _cores(),
+            "kind": "oracle",
+            "sample": f"{nr} of 4680 query rows of each of the 5 nodes, all 12 heads, full key "
+                      f"lists ({flops / 1e9:.1f} GFLOP in {dt:.2f} s, float64 numpy)"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    active, entries, qs = _oracle_round()
+    n_rows = 24
+    for _ in range(args.warmup):
+        _oracle_sample(active, entries, qs, n_rows)
+    times, flops = [], 0
+    for _ in range(args.steps):
+        dt, flops, nr = _oracle_sample(active, entries, qs, n_rows)
+        times.append(dt)
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / len(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference", "config": _config(),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _cores(),
+                         "kind": "oracle",
+                         "sample": f"{nr} of 4680 query rows per node per step, all heads, "
+                                   "full key lists"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["wave", "reference"], default="wave")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

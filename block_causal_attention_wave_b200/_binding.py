@@ -1,0 +1,242 @@
+"""ctypes binding of libwave.so: argument marshalling only.
+
+Every computation (scheduling, page allocation, key tables, the append and
+attention kernels) happens inside the C library; this module turns Python
+values and torch tensors into the plain pointers and sizes the C ABI takes.
+There is no fallback: if the library is missing, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwave.so")
+
+OK = 0
+ERR_ARG, ERR_MISSING_KV, ERR_NO_PAGES, ERR_CUDA = -1, -2, -3, -4
+ERR_TIMEOUT, ERR_EXISTS, ERR_CAPACITY, ERR_UNSUPPORTED = -5, -6, -7, -8
+POLICIES = {"clean": 0, "same": 1, "progressive": 2}
+PAGE_TOKENS = 128
+PREFIX_CHUNK = -1
+MAX_NODES = 64
+MAX_PAGES_PER_ROUND = 7168
+
+_lib = None
+
+
+class WaveError(RuntimeError):
+    def __init__(self, code: int, detail: str):
+        super().__init__(f"wave error {code}: {detail}")
+        self.code = code
+
+
+class Node(ctypes.Structure):
+    _fields_ = [("chunk", ctypes.c_int32), ("level", ctypes.c_int32)]
+
+
+class KVConfig(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("tokens_per_chunk", ctypes.c_int32), ("num_levels", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("prefix_tokens", ctypes.c_int32),
+                ("pool", ctypes.c_void_p), ("pool_bytes", ctypes.c_uint64)]
+
+
+_SIGS = {
+    "wave_kv_create": (ctypes.c_int, [ctypes.POINTER(KVConfig), ctypes.POINTER(ctypes.c_void_p)]),
+    "wave_kv_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "wave_kv_pool_layout": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64),
+                                           ctypes.POINTER(ctypes.c_int64),
+                                           ctypes.POINTER(ctypes.c_int32)]),
+    "wave_kv_alloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32]),
+    "wave_kv_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                      ctypes.c_void_p]),
+    "wave_kv_release": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32]),
+    "wave_kv_free_pages": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)]),
+    "wave_gather_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                         ctypes.POINTER(ctypes.c_int32)]),
+    "wave_round_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p]),
+    "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.POINTER(Node), ctypes.c_int32,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                     ctypes.POINTER(ctypes.c_int32),
+                                     ctypes.POINTER(ctypes.c_int32)]),
+    "wave_schedule_last_read": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_int32, ctypes.POINTER(Node),
+                                               ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
+    "wave_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "wave_last_error_detail": (ctypes.c_char_p, []),
+}
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libwave.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m block_causal_attention_wave_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _check(rc: int):
+    if rc != OK:
+        detail = _lib.wave_last_error_detail().decode() or _lib.wave_strerror(rc).decode()
+        raise WaveError(rc, detail)
+
+
+def _policy(policy) -> int:
+    return POLICIES[policy] if isinstance(policy, str) else int(policy)
+
+
+def _nodes(active):
+    arr = (Node * max(1, len(active)))()
+    for i, (c, l) in enumerate(active):
+        arr[i].chunk, arr[i].level = int(c), int(l)
+    return arr
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def schedule(B: int, K: int, policy="progressive", window: int = 0):
+    """Rounds of (chunk, level) nodes, as computed by the library."""
+    lib = load()
+    nn, nr = ctypes.c_int32(0), ctypes.c_int32(0)
+    rc = lib.wave_schedule(B, K, _policy(policy), window, None, 0, None, 0,
+                           ctypes.byref(nn), ctypes.byref(nr))
+    if rc not in (OK, ERR_CAPACITY):
+        _check(rc)
+    nodes = (Node * nn.value)()
+    offs = (ctypes.c_int32 * (nr.value + 1))()
+    _check(lib.wave_schedule(B, K, _policy(policy), window, nodes, nn.value, offs, nr.value + 1,
+                             ctypes.byref(nn), ctypes.byref(nr)))
+    return [[(nodes[i].chunk, nodes[i].level) for i in range(offs[t], offs[t + 1])]
+            for t in range(nr.value)]
+
+
+def last_read_rounds(B: int, K: int, policy="progressive", window: int = 0, nodes=None):
+    """Dict (chunk, level) -> last round reading that entry, from the library."""
+    lib = load()
+    if nodes is None:
+        nodes = [n for r in schedule(B, K, policy, window) for n in r]
+    arr = _nodes(nodes)
+    out = (ctypes.c_int32 * max(1, len(nodes)))()
+    _check(lib.wave_schedule_last_read(B, K, _policy(policy), window, arr, len(nodes), out))
+    return {tuple(n): out[i] for i, n in enumerate(nodes)}
+
+
+class KVCache:
+    """Handle on a paged (chunk, level) K/V pool.
+
+    ``pool`` is a caller-owned CUDA uint8 tensor (kept alive by this object).
+    With ``pool=None`` the handle is host-only: allocation and tables work,
+    kernels do not; ``pool_bytes`` then sets the page count.
+    """
+
+    def __init__(self, heads, head_dim, tokens_per_chunk, num_levels, window=0,
+                 prefix_tokens=0, pool=None, pool_bytes=None):
+        self.lib = load()
+        self.heads, self.head_dim = heads, head_dim
+        self.tokens, self.levels = tokens_per_chunk, num_levels
+        self.window, self.prefix_tokens = window, prefix_tokens
+        self.pool = pool
+        if pool is not None:
+            pool_bytes = pool.numel() * pool.element_size()
+            ptr = pool.data_ptr()
+        else:
+            ptr = None
+        cfg = KVConfig(heads, head_dim, tokens_per_chunk, num_levels, window, prefix_tokens,
+                       ptr, int(pool_bytes))
+        h = ctypes.c_void_p()
+        _check(self.lib.wave_kv_create(ctypes.byref(cfg), ctypes.byref(h)))
+        self.h = h
+
+    @staticmethod
+    def page_bytes(heads, head_dim) -> int:
+        return 2 * heads * PAGE_TOKENS * head_dim * 2
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.wave_kv_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def layout(self):
+        pb, off, mp = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+        _check(self.lib.wave_kv_pool_layout(self.h, ctypes.byref(pb), ctypes.byref(off),
+                                            ctypes.byref(mp)))
+        return pb.value, off.value, mp.value
+
+    def alloc(self, chunk, level, ntokens=None):
+        n = self.tokens if ntokens is None else ntokens
+        _check(self.lib.wave_kv_alloc(self.h, chunk, level, n))
+
+    def append(self, chunk, level, K, V, stream=None):
+        n = K.shape[0]
+        _check(self.lib.wave_kv_append(self.h, chunk, level, ctypes.c_void_p(K.data_ptr()),
+                                       ctypes.c_void_p(V.data_ptr()), n, _stream_handle(stream)))
+
+    def release(self, chunk, level):
+        _check(self.lib.wave_kv_release(self.h, chunk, level))
+
+    def free_pages(self) -> int:
+        n = ctypes.c_int32()
+        _check(self.lib.wave_kv_free_pages(self.h, ctypes.byref(n)))
+        return n.value
+
+    def gather_table(self, active, policy):
+        """Per node, a list of (page id, valid tokens) in key order."""
+        nodes = _nodes(active)
+        n = ctypes.c_int32()
+        rc = self.lib.wave_gather_table(self.h, nodes, len(active), _policy(policy), None, None, 0,
+                                        ctypes.byref(n))
+        if rc not in (OK, ERR_CAPACITY):
+            _check(rc)
+        rows = (ctypes.c_int32 * (2 * max(1, n.value)))()
+        offs = (ctypes.c_int32 * (len(active) + 1))()
+        _check(self.lib.wave_gather_table(self.h, nodes, len(active), _policy(policy), rows, offs,
+                                          n.value, ctypes.byref(n)))
+        return [[(rows[2 * r], rows[2 * r + 1]) for r in range(offs[i], offs[i + 1])]
+                for i in range(len(active))]
+
+    def round_attn(self, active, policy, Q, O, stream=None):
+        """O[i*T:(i+1)*T] = attention of active node i over its key list."""
+        nodes = _nodes(active)
+        _check(self.lib.wave_round_attn(self.h, nodes, len(active), _policy(policy),
+                                        ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(O.data_ptr()),
+                                        _stream_handle(stream)))
+        return O
+
+    def status(self, stream=None):
+        """Synchronise and raise WaveError if a kernel timed out."""
+        _check(self.lib.wave_kv_status(self.h, _stream_handle(stream)))

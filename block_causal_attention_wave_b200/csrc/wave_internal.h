@@ -1,0 +1,63 @@
+// Internal declarations shared by the host (wave_host.cpp) and device (*.cu)
+// halves of libwave.so. Not part of the ABI.
+#pragma once
+
+#include <cuda.h>  // CUtensorMap (type only; the driver is reached at run time)
+
+#include <cstdint>
+#include <map>
+#include <set>
+#include <utility>
+#include <vector>
+
+#include "wave.h"
+
+struct wave_entry {
+  std::vector<int32_t> pages;  // page ids in token order
+  int32_t ntokens = 0;
+};
+
+struct wave_kv {
+  wave_kv_config cfg{};
+  int64_t page_bytes = 0;   // 2 * H * 128 * d * sizeof(bf16)
+  int64_t data_offset = 0;  // byte offset of page 0 inside the pool
+  int32_t max_pages = 0;
+  std::set<int32_t> free_pages;  // ordered: begin() is the lowest free id
+  std::map<std::pair<int32_t, int32_t>, wave_entry> entries;
+  bool on_device = false;  // pool != NULL
+  int device = -1;
+  int num_sms = 0;
+  alignas(64) CUtensorMap tm_kv;  // rows of d bf16 over every page's K and V
+};
+
+namespace wavei {
+
+constexpr int kPageTokens = WAVE_PAGE_TOKENS;
+constexpr int64_t kHeaderBytes = 4096;  // device status word lives here
+
+// Record a message for wave_last_error_detail() and return `code`.
+int fail(int code, const char* fmt, ...);
+void clear_error();
+
+// phi(j, r) of the design-space paper, Table 1 (r >= 1).
+int phi(int policy, int j, int r);
+bool valid_policy(int policy);
+
+// Ordered entries (chunk, level) of a node's key list: prefix, history by
+// ascending chunk, own entry.
+void key_entries(const wave_kv* kv, wave_node node, int policy,
+                 std::vector<std::pair<int32_t, int32_t>>& out);
+
+// Per active node, its (page, valid) rows; offsets has n + 1 entries.
+int build_rows(const wave_kv* kv, const wave_node* active, int n, int policy,
+               std::vector<int32_t>& rows, std::vector<int32_t>& offsets);
+
+// Validate one query node against the handle's shape.
+int check_query_node(const wave_kv* kv, wave_node node);
+
+// Device halves (defined in .cu files).
+int device_init(wave_kv* kv);
+int launch_append(wave_kv* kv, const wave_entry& e, const void* K, const void* V,
+                  int32_t ntokens, void* stream);
+
+}  // namespace wavei

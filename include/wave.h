@@ -1,0 +1,188 @@
+/*
+ * wave.h -- C ABI of the wave-round block-causal attention library (libwave.so).
+ *
+ * The method: pipelined streaming video diffusion. In one concurrent forward
+ * round several chunks sit at staggered denoising levels; each attends to its
+ * own tokens plus the K/V of earlier chunks at the levels a context policy
+ * phi(j, r) picks (level 0 = clean). Sources, cited by page title and section:
+ *   [WF]  "Wave Forcing: towards speed-of-light streaming video generation"
+ *         (aiany.app), "Key Findings": one output chunk per concurrent round,
+ *         chunk-wise causal attention over earlier cleaner chunks, cache
+ *         refresh, early K/V delivery.
+ *   [DS]  design-space paper (thelatestinai.com, arXiv 2609.22283 summary),
+ *         Table 1 and Figure 1 (policies), Figure 2 (serial B*K vs pipelined
+ *         B+K-1 rounds), Appendix Table 4 (7 chunks of 3 latent frames).
+ *   [WS]  "Wan-Streamer v0.2: Higher Resolution, Same Latency", Figure 1 and
+ *         glossary "block-causal attention", "K/V cache", "pre-sharded".
+ *
+ * Conventions for every call:
+ *   - Returns WAVE_OK (0) or a negative WAVE_ERR_* code; nothing throws across
+ *     the ABI. wave_strerror() names a code; wave_last_error_detail() gives a
+ *     message for the last failure on the calling thread.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Device work is enqueued on it and is asynchronous; inputs must stay valid
+ *     and unmodified until that work has run.
+ *   - Device buffers are caller-owned. The library never calls cudaMalloc; the
+ *     K/V pool is one caller-provided device buffer (see wave_kv_config).
+ *   - Activations are bf16, token-major and contiguous: [tokens][heads][head_dim].
+ *   - No call is thread-safe on the same wave_kv handle.
+ */
+#ifndef WAVE_H_
+#define WAVE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define WAVE_OK               0
+#define WAVE_ERR_ARG         (-1) /* bad argument, shape or alignment            */
+#define WAVE_ERR_MISSING_KV  (-2) /* a (chunk, level) the policy reads is absent */
+#define WAVE_ERR_NO_PAGES    (-3) /* the pool has too few free pages             */
+#define WAVE_ERR_CUDA        (-4) /* a CUDA runtime/driver call failed           */
+#define WAVE_ERR_TIMEOUT     (-5) /* a kernel's bounded wait ran out             */
+#define WAVE_ERR_EXISTS      (-6) /* (chunk, level) already holds K/V            */
+#define WAVE_ERR_CAPACITY    (-7) /* a round exceeds one launch's table limits   */
+#define WAVE_ERR_UNSUPPORTED (-8) /* head_dim or device not supported            */
+
+/* ---- context policies phi(j, r) ([DS] Table 1, Figure 1) ---------------- */
+#define WAVE_POLICY_CLEAN       0 /* phi = 0                */
+#define WAVE_POLICY_SAME        1 /* phi = j                */
+#define WAVE_POLICY_PROGRESSIVE 2 /* phi = max(j - r, 0)    */
+
+#define WAVE_PAGE_TOKENS   128   /* tokens per K/V page                       */
+#define WAVE_PREFIX_CHUNK  (-1)  /* chunk id of the always-visible prefix     */
+#define WAVE_MAX_NODES     64    /* active nodes per wave_round_attn call     */
+#define WAVE_MAX_PAGES_PER_ROUND 7168 /* key pages summed over a call's nodes */
+
+typedef struct wave_kv wave_kv; /* opaque; owned by the library */
+
+/* One (chunk, level) node. Level 0 = clean; an update at level j >= 1 turns the
+ * level-j state into level j-1; a level-0 node is a cache refresh ([WF]). */
+typedef struct {
+  int32_t chunk;
+  int32_t level;
+} wave_node;
+
+typedef struct {
+  int32_t heads;            /* H (query heads = K/V heads)                        */
+  int32_t head_dim;         /* d: 64 or 128                                       */
+  int32_t tokens_per_chunk; /* T: tokens of one chunk / streaming unit            */
+  int32_t num_levels;       /* K: update levels K..1                               */
+  int32_t window;           /* W: history chunks visible; 0 = unbounded           */
+  int32_t prefix_tokens;    /* conditioning prefix length; 0 = none               */
+  void*    pool;            /* caller-owned device buffer, 256-byte aligned, or
+                               NULL for a host-only handle (tables, no kernels)   */
+  uint64_t pool_bytes;      /* size of pool (for a host-only handle: the size the
+                               page count is derived from)                       */
+} wave_kv_config;
+
+/* Create a paged (chunk, level) K/V cache over cfg->pool ([WF] history cache,
+ * [WS] "K/V cache"). The pool holds a 4096-byte header (device status word)
+ * followed by pages of 2*H*128*d bf16 values: K as [H][128][d], then V as
+ * [H][128][d]. Page p starts at pool + data_offset + p * page_bytes. With a
+ * non-NULL pool this call clears the header synchronously and needs a CUDA
+ * device with sm_100. *out receives the handle; destroy it with
+ * wave_kv_destroy. Errors: ARG (bad sizes, misaligned pool, pool too small),
+ * UNSUPPORTED (head_dim not 64/128, or a device other than sm_100), CUDA. */
+int wave_kv_create(const wave_kv_config* cfg, wave_kv** out);
+
+/* Destroy a handle (the pool stays the caller's). NULL is accepted. */
+int wave_kv_destroy(wave_kv* kv);
+
+/* Report the pool layout: bytes per page, byte offset of page 0, page count. */
+int wave_kv_pool_layout(const wave_kv* kv, int64_t* page_bytes, int64_t* data_offset,
+                        int32_t* max_pages);
+
+/* Reserve pages for entry (chunk, level) holding ntokens tokens without
+ * writing them: ceil(ntokens/128) pages, each the lowest free page id, taken
+ * in call order. chunk = WAVE_PREFIX_CHUNK (level 0) names the prefix, whose
+ * ntokens must equal prefix_tokens; any other chunk needs ntokens =
+ * tokens_per_chunk and 0 <= level <= num_levels. Host only, no device work.
+ * Errors: ARG, EXISTS, NO_PAGES (nothing is taken then). */
+int wave_kv_alloc(wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens);
+
+/* wave_kv_alloc, then copy K and V (device, bf16 [ntokens][H][d], contiguous,
+ * 16-byte aligned, caller-owned) into the new pages with one kernel on stream;
+ * the unused tail of the last page is zero-filled. This is the in-round K/V
+ * delivery of [WF] and the local-cache write of [WS] "pre-sharded".
+ * Errors: as wave_kv_alloc, plus ARG for misaligned K/V and CUDA; on any error
+ * no pages stay taken. */
+int wave_kv_append(wave_kv* kv, int32_t chunk, int32_t level, const void* K, const void* V,
+                   int32_t ntokens, void* stream);
+
+/* Return the pages of (chunk, level) to the free set. Host only; the caller
+ * must not release an entry that queued device work still reads (all library
+ * kernels read the pool in stream order, so releasing after enqueueing the
+ * last reader on the same stream is safe when the next writer uses that
+ * stream too). Errors: MISSING_KV. */
+int wave_kv_release(wave_kv* kv, int32_t chunk, int32_t level);
+
+/* Number of free pages. */
+int wave_kv_free_pages(const wave_kv* kv, int32_t* n);
+
+/* The key list of each active node, as the attention kernel reads it: for node
+ * i, rows node_offsets[i] .. node_offsets[i+1]-1 of `rows`, each row a pair
+ * (page id, valid tokens) = rows[2*r], rows[2*r+1]. Key order: prefix, then
+ * history E(c - r, phi(l, r)) for r = min(c, W)..1 (ascending chunk), then the
+ * node's own E(c, l) ([DS] Table 1; [WF] "Key Findings"). `cap` = capacity of
+ * rows in pairs; node_offsets holds n_active + 1 ints. Host only.
+ * Errors: ARG, MISSING_KV, CAPACITY (cap too small; *n_rows = pairs needed). */
+int wave_gather_table(const wave_kv* kv, const wave_node* active, int32_t n_active,
+                      int32_t policy, int32_t* rows, int32_t* node_offsets, int32_t cap,
+                      int32_t* n_rows);
+
+/* One wave round of block-causal attention for all active nodes in ONE kernel
+ * launch: for node i = (c, l) and head h,
+ *   O_i[q, h] = softmax_k(Q_i[q, h] . K[k, h] / sqrt(d)) V[k, h]
+ * over the tokens of the node's key list (see wave_gather_table); no mask
+ * inside a chunk ([WS] "block-causal attention"; [DS] Figure 1).
+ * Q and O: device bf16 [n_active * T][H][d], node i's rows at i*T, 16-byte
+ * aligned, caller-owned; O is written, Q is read. Every entry the nodes read
+ * must have been appended (on this stream or before it). Accumulation is fp32;
+ * O is rounded to bf16 once. Limits: n_active <= WAVE_MAX_NODES, total key
+ * pages <= WAVE_MAX_PAGES_PER_ROUND (else CAPACITY). A device-side timeout is
+ * reported by the next wave_kv_status call. Errors: ARG, MISSING_KV, CAPACITY,
+ * CUDA. */
+int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
+                    const void* Q, void* O, void* stream);
+
+/* Synchronise `stream`, then read and clear the pool's device status word.
+ * Returns WAVE_OK, WAVE_ERR_TIMEOUT if a kernel gave up on a bounded wait
+ * (its output is then undefined), or WAVE_ERR_CUDA. */
+int wave_kv_status(wave_kv* kv, void* stream);
+
+/* Round schedule for B chunks and K levels under `policy` and `window`
+ * ([DS] Figure 2; [WF] "Key Findings"). Nodes: updates (c, j), j = K..1, and
+ * refreshes (c, 0) where some node reads E(c, 0). Node (c, l) reads E(c, l)
+ * and E(c - r, phi(l, r)) for r = 1..min(c, W). Each node runs in the least
+ * round with round(c, l) >= round(c, l+1) + 1, round(c, K) >= c, and
+ * round >= the round that writes each entry it reads (K/V written in a round
+ * is visible in that round). Output: round t holds nodes
+ * [round_offsets[t], round_offsets[t+1]) of `nodes`, ascending chunk.
+ * Progressive and same-level give B+K-1 rounds, clean gives B*K.
+ * Errors: ARG, CAPACITY (caps too small; *n_nodes, *n_rounds = sizes needed). */
+int wave_schedule(int32_t B, int32_t K, int32_t policy, int32_t window, wave_node* nodes,
+                  int32_t nodes_cap, int32_t* round_offsets, int32_t rounds_cap,
+                  int32_t* n_nodes, int32_t* n_rounds);
+
+/* Last round in which any node of the (B, K, policy, window) schedule reads
+ * the entry E(c, l) of each given node (its own round at least). A rollout
+ * driver releases E(c, l) after that round's attention. Host only.
+ * Errors: ARG (bad sizes, or a node that is not in the schedule). */
+int wave_schedule_last_read(int32_t B, int32_t K, int32_t policy, int32_t window,
+                            const wave_node* nodes, int32_t n, int32_t* last_round);
+
+/* Static name of a status code. */
+const char* wave_strerror(int code);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* wave_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WAVE_H_ */

@@ -1,0 +1,212 @@
+"""GPU parity: libwave.so's append and attention kernels vs the float64 oracle.
+
+Every test here runs the CUDA path through the C ABI and compares with the
+oracle on the same seeded bf16 inputs: element by element on small cases that
+span several query tiles, several pages and ragged tails; on sampled query rows
+at the full workload sizes (Wan2.1 round, Wan-Streamer unit, long rollout).
+Bar: max-abs <= 1e-2 and relative L2 <= 5e-3 per node; gather tables and the
+appended page bytes bit-exact.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import wave_inputs as wi
+from oracle import cache as ocache
+from oracle import schedule as osched
+
+from wave_testlib import (Inputs, append, assert_close, bits_to_torch, make_cache, oracle_outputs,
+                          queries, torch_to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _rollout_and_check(wave, wl, pol, check_rounds=None, rows_per_node=None, pages=4000):
+    """Drive a full rollout through the library; check outputs and tables."""
+    import torch
+    inp = Inputs(wl)
+    kv = make_cache(wave, wl, pages)
+    rounds = wave.schedule(wl.chunks, wl.levels, pol, wl.window)
+    last = wave.last_read_rounds(wl.chunks, wl.levels, pol, wl.window)
+    want_tables = ocache.rollout_tables(wl.chunks, wl.levels, pol, wl.window, wl.tokens,
+                                        wl.prefix, kv.layout()[2])
+    if wl.prefix:
+        append(kv, inp, (-1, 0))
+    keep = []
+    results = []
+    for t, active in enumerate(rounds):
+        for n in active:
+            keep.append(append(kv, inp, n))
+        assert kv.gather_table(active, pol) == want_tables[t][1], f"round {t} table"
+        if check_rounds is None or t in check_rounds:
+            q = queries(inp, active)
+            o = torch.empty_like(q)
+            kv.round_attn(active, pol, q, o)
+            kv.status()
+            rows = None
+            if rows_per_node is not None:
+                rows = {n: rows_per_node for n in active}
+            ref = oracle_outputs(inp, active, pol, rows)
+            got = torch_to_f64(o).reshape(len(active), wl.tokens, wl.heads, wl.head_dim)
+            for i, n in enumerate(active):
+                g = got[i] if rows is None else got[i][rows[n]]
+                results.append(assert_close(g, ref[n], f"{wl.name} {pol} round {t} node {n}"))
+        for e in sorted(e for e, lr in last.items() if lr == t):
+            kv.release(*e)
+    torch.cuda.synchronize()
+    return results
+
+
+@pytest.mark.parametrize("pol", wi.POLICIES)
+def test_tiny_all_rounds(cuda_lib, pol):
+    """Tiny case: 3 chunks, 2 levels, 2 heads, d 64, 32 tokens; every round."""
+    _rollout_and_check(cuda_lib, wi.TINY, pol)
+
+
+SMALL = [
+    wi.Workload("small-d128", chunks=4, levels=3, heads=3, head_dim=128, tokens=300),
+    wi.Workload("small-d64-prefix-window", chunks=5, levels=2, heads=2, head_dim=64, tokens=260,
+                window=2, prefix=200),
+    wi.Workload("small-d128-prefix", chunks=3, levels=2, heads=2, head_dim=128, tokens=128,
+                prefix=77),
+    wi.Workload("small-k1", chunks=4, levels=1, heads=2, head_dim=128, tokens=129),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("pol", wi.POLICIES)
+def test_small_multi_tile_ragged(cuda_lib, wl, pol):
+    """Several query tiles and pages with ragged tails; every round, every element."""
+    _rollout_and_check(cuda_lib, wl, pol)
+
+
+def test_append_bytes_exact(cuda_lib):
+    """Pages hold exactly the appended K/V in [H][128][d] order, tail zero."""
+    import torch
+    wl = wi.Workload("append", chunks=2, levels=1, heads=3, head_dim=128, tokens=300)
+    inp = Inputs(wl)
+    kv = make_cache(cuda_lib, wl, 16)
+    kv.alloc(0, 1)  # occupy pages 0..2 so the appended entry starts at page 3
+    append(kv, inp, (1, 1))
+    (rows,) = kv.gather_table([(1, 1)], "same")
+    torch.cuda.synchronize()
+    page_bytes, off, _ = kv.layout()
+    pool = kv.pool.cpu().numpy()
+    tail = 1
+    for kind, kvi in (("k", 0), ("v", 1)):
+        src = inp.bits(kind, 1, 1)  # [T][H][d]
+        for pi, (page, valid) in enumerate(rows[-3:]):
+            base = off + page * page_bytes + kvi * wl.heads * 128 * wl.head_dim * 2
+            blk = pool[base:base + wl.heads * 128 * wl.head_dim * 2].view(np.uint16)
+            blk = blk.reshape(wl.heads, 128, wl.head_dim)
+            want = np.zeros_like(blk)
+            n = min(128, wl.tokens - pi * 128)
+            want[:, :n, :] = src[pi * 128:pi * 128 + n].transpose(1, 0, 2)
+            np.testing.assert_array_equal(blk, want)
+            tail = valid
+    assert tail == 300 - 256
+
+
+@pytest.mark.parametrize("pol", ["progressive", "clean"])
+def test_wan21_round6_sampled_rows(cuda_lib, pol):
+    """Full Wan2.1-shaped round (12 heads, d 128, 4680 tokens), sampled query rows."""
+    wl = wi.WAN21
+    rounds = osched.schedule(wl.chunks, wl.levels, pol)
+    t_check = 6 if pol == "progressive" else 10
+    rows = np.array([0, 1, 127, 128, 1000, 2047, 2048, 3333, 4607, 4608, 4650, 4679])
+    res = _rollout_and_check(cuda_lib, wl, pol, check_rounds={t_check}, rows_per_node=rows,
+                             pages=1200)
+    assert len(res) == len(rounds[t_check])
+
+
+def _one_round(wave, wl, pol, t, rows):
+    """Append just what round t reads, run it, compare sampled rows."""
+    import torch
+    inp = Inputs(wl)
+    rounds = osched.schedule(wl.chunks, wl.levels, pol, wl.window)
+    active = rounds[t]
+    needed = set()
+    for n in active:
+        needed.update(ocache.key_entries(n, pol, wl.window, wl.prefix > 0))
+    per_entry = ocache.pages_for(max(wl.tokens, wl.prefix))
+    kv = make_cache(wave, wl, len(needed) * per_entry + 8)
+    keep = [append(kv, inp, e) for e in sorted(needed)]
+    q = queries(inp, active)
+    o = torch.empty_like(q)
+    kv.round_attn(active, pol, q, o)
+    kv.status()
+    ref = oracle_outputs(inp, active, pol, {n: rows for n in active})
+    got = torch_to_f64(o).reshape(len(active), wl.tokens, wl.heads, wl.head_dim)
+    del keep
+    return [assert_close(got[i][rows], ref[n], f"{wl.name} round {t} node {n}")
+            for i, n in enumerate(active)]
+
+
+def test_wan_streamer_steady_round(cuda_lib):
+    """Wan-Streamer-shaped unit: 24 heads, 984 tokens, 512 prefix, 32-unit window."""
+    rows = np.array([0, 5, 127, 128, 500, 895, 896, 983])
+    res = _one_round(cuda_lib, wi.WAN_STREAMER, "progressive", 35, rows)
+    assert len(res) == 3
+
+
+def test_long_rollout_steady_round(cuda_lib):
+    """40 chunks x 4680 tokens, window 6, 5 levels: a steady-state round."""
+    rows = np.array([0, 77, 128, 2500, 4608, 4679])
+    res = _one_round(cuda_lib, wi.LONG_ROLLOUT, "progressive", 20, rows)
+    assert len(res) == 6
+
+
+def test_same_level_max_growth_rescales(cuda_lib):
+    """Scores that grow along the key list force the O rescale path."""
+    import torch
+    wl = wi.Workload("growth", chunks=3, levels=1, heads=2, head_dim=128, tokens=256)
+    inp = Inputs(wl)
+    # Scale each entry's K by a growing factor so later pages carry larger scores.
+    for c, f in ((0, 0.25), (1, 1.0), (2, 4.0)):
+        kb = inp.bits("k", c, 1)
+        kf = wi.bf16_bits_to_f64(kb) * f
+        inp._bits[("k", c, 1)] = wi.f32_to_bf16_bits(kf.astype(np.float32))
+    kv = make_cache(cuda_lib, wl, 32)
+    keep = [append(kv, inp, (c, 1)) for c in range(3)]
+    active = [(2, 1)]
+    q = queries(inp, active)
+    o = torch.empty_like(q)
+    kv.round_attn(active, "same", q, o)
+    kv.status()
+    ref = oracle_outputs(inp, active, "same")
+    assert float(np.abs(ref[(2, 1)]).max()) > 1.0  # outputs well above 1: bf16 ulp matters
+    assert_close(torch_to_f64(o), ref[(2, 1)], "growth", scale_with_output=True)
+    del keep
+
+
+def test_missing_kv_is_reported_before_launch(cuda_lib):
+    import torch
+    wl = wi.TINY
+    kv = make_cache(cuda_lib, wl, 8)
+    inp = Inputs(wl)
+    keep = append(kv, inp, (1, 2))
+    q = queries(inp, [(1, 2)])
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.round_attn([(1, 2)], "progressive", q, torch.empty_like(q))
+    assert e.value.code == -2
+    kv.status()
+    del keep
+
+
+def test_duplicate_and_single_nodes(cuda_lib):
+    """The same node twice in one launch gives the same rows twice."""
+    import torch
+    wl = dataclasses.replace(wi.TINY, tokens=200, head_dim=128)
+    inp = Inputs(wl)
+    kv = make_cache(cuda_lib, wl, 16)
+    keep = [append(kv, inp, e) for e in ((0, 0), (1, 1))]
+    active = [(1, 1), (1, 1)]
+    q = queries(inp, active)
+    o = torch.empty_like(q)
+    kv.round_attn(active, "progressive", q, o)
+    kv.status()
+    assert torch.equal(o[:200], o[200:])
+    ref = oracle_outputs(inp, [(1, 1)], "progressive")
+    assert_close(torch_to_f64(o[:200]), ref[(1, 1)], "dup")
+    del keep
