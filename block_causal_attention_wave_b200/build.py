@@ -42,7 +42,7 @@ def build(verbose_ptxas: bool = False, out: str = LIB) -> str:
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc()] + common + ["-c", src, "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
         if r.returncode != 0 or verbose_ptxas:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:
@@ -50,7 +50,7 @@ def build(verbose_ptxas: bool = False, out: str = LIB) -> str:
         objs.append(obj)
     tmp = out + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
-    r = subprocess.run(cmd, capture_output=True, text=True)
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link of libwave.so failed")

@@ -41,6 +41,7 @@
 #include <numeric>
 #include <vector>
 
+#include "exp2_poly.h"
 #include "ptx.cuh"
 #include "wave_internal.h"
 
@@ -50,7 +51,15 @@ namespace wavei {
 
 namespace {
 
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 softmax (2 groups)
+// Register split after start-up (setmaxnreg): warps 0..3 (TMA, MMA, two idle;
+// one per SM sub-partition) drop to kRegsLow, the two softmax warpgroups (two
+// warps per sub-partition) rise to kRegsHigh, so each softmax thread can hold
+// a full 128-column S row. Per sub-partition 88 + 2 x 208 = 504 <= 512
+// registers per lane, i.e. the sum equals what the launch holds at 168 per
+// thread; the host refuses to launch a build compiled with fewer.
+constexpr uint32_t kRegsLow = 88, kRegsHigh = 208, kRegsLaunch = 168;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 constexpr uint32_t kPageMask = (1u << 25) - 1;  // page id bits of a page word
@@ -60,7 +69,7 @@ struct AttnNode {
   int32_t page0;     // first page word
   int32_t n_pages;   // key pages
   int32_t item0;     // first work item
-  int32_t n_qtiles;  // ceil(T / 128)
+  int32_t n_pairs;   // ceil(ceil(T / 128) / 2): pairs of 128-row query tiles
   int32_t pad;
 };
 
@@ -80,19 +89,23 @@ struct AttnParams {
 };
 static_assert(sizeof(AttnParams) <= 32760, "kernel parameter space is 32 KB");
 
+// Softmax columns (of each 32) whose exp2 runs on the FMA pipe (polynomial)
+// instead of the special-function unit.
+constexpr int kEmuPerChunk = 8;
+
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;           // 64-column, 128-byte-wide panels
   static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = 128 * D * 2;   // one Q, K or V tile
-  static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
-  // TMEM columns: S0, S1 (128 fp32 each), O (d fp32), P0, P1 (64 x bf16x2 each).
-  static constexpr uint32_t kColS = 0, kColO = 256, kColP = 384, kCols = 512;
+  static constexpr int kSlots = D == 128 ? 5 : 10; // K/V ring slots (K and V alternate)
+  static constexpr int kQOff = 0;                  // Q0, then Q1
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
+  // TMEM columns: S_w at 128 w (fp32; P_w as bf16x2 overwrites its first 64
+  // columns), O_w at 256 + 128 w.
+  static constexpr uint32_t kColS = 0, kColO = 256, kCols = 512;
   // Instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128.
   static constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
                                       ((128u >> 4) << 24);
@@ -104,21 +117,20 @@ struct Cfg {
 enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
-  B_S_FULL,        // 2
-  B_P_FULL = B_S_FULL + 2,  // 2
-  B_PV_DONE = B_P_FULL + 2,
-  B_O_FULL,
-  B_O_EMPTY,
-  B_DRAIN,
-  B_K_FULL,        // kStages each from here
+  B_S_FULL,                 // 2: S_w computed
+  B_P_FULL = B_S_FULL + 2,  // 2: P_w written (128 arrivals)
+  B_O_FULL = B_P_FULL + 2,  // 2: last P.V of an item done
+  B_O_EMPTY = B_O_FULL + 2, // 2: epilogue has read O_w (128 arrivals)
+  B_DRAIN = B_O_EMPTY + 2,
+  B_RING_FULL,              // kSlots each from here
 };
 
 template <int D>
 struct Bars {
-  static constexpr int kS = Cfg<D>::kStages;
-  static constexpr int K_FULL = B_K_FULL, K_EMPTY = K_FULL + kS, V_FULL = K_EMPTY + kS,
-                       V_EMPTY = V_FULL + kS, COUNT = V_EMPTY + kS;
-  static_assert(COUNT * 8 + 16 <= 256, "barrier area");
+  static constexpr int kS = Cfg<D>::kSlots;
+  static constexpr int RING_FULL = B_RING_FULL, RING_EMPTY = RING_FULL + kS,
+                       COUNT = RING_EMPTY + kS;
+  static_assert(COUNT * 8 + 16 <= 512, "barrier area");
 };
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
@@ -138,7 +150,7 @@ struct Ctl {
 };
 
 // Bounded wait on an mbarrier phase. Returns false if this CTA is stopping.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& ctl, int code) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& ctl, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
@@ -155,22 +167,46 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& 
 
 // Bounded wait that ignores the stop flag: used only while stopping, to let
 // asynchronous copies or MMAs that were already issued complete.
-__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > kDrainNs) return;
 }
 
 struct Item {
-  int node, head, qtile;
+  int node, head, pair;
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   int n = 0;
   while (n + 1 < p.n_nodes && item >= p.nodes[n + 1].item0) ++n;
   const int j = item - p.nodes[n].item0;
-  const int nq = p.nodes[n].n_qtiles;
-  return Item{n, j / nq, j % nq};
+  const int np = p.nodes[n].n_pairs;
+  return Item{n, j / np, j % np};
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe: x = j + f, j = round(x),
+// |f| <= 1/2, 2^f from the minimax cubic of exp2_poly.h, 2^j added to the
+// exponent field. Inputs below -126 (including -inf) are clamped there, giving
+// at most 2^-126 -- negligible against a row sum >= 1.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t jf = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(WAVE_EXP2_C3, WAVE_EXP2_C3), f, f2_pack(WAVE_EXP2_C2, WAVE_EXP2_C2));
+  p = f2_fma(p, f, f2_pack(WAVE_EXP2_C1, WAVE_EXP2_C1));
+  p = f2_fma(p, f, f2_pack(WAVE_EXP2_C0, WAVE_EXP2_C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // The low mantissa bits of t hold j (two's complement); shifting them into
+  // the exponent field scales p by 2^j.
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 template <int D>
@@ -178,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     round_attn_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   using BR = Bars<D>;
-  constexpr int S = C::kStages;
+  constexpr int S = C::kSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -194,19 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_EMPTY), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(B_S_FULL + b), 1);
-      mbar_init(bar(B_P_FULL + b), 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(B_S_FULL + w), 1);
+      mbar_init(bar(B_P_FULL + w), 128);
+      mbar_init(bar(B_O_FULL + w), 1);
+      mbar_init(bar(B_O_EMPTY + w), 128);
     }
-    mbar_init(bar(B_PV_DONE), 1);
-    mbar_init(bar(B_O_FULL), 1);
-    mbar_init(bar(B_O_EMPTY), 128);
     mbar_init(bar(B_DRAIN), 1);
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(BR::K_FULL + s), 1);
-      mbar_init(bar(BR::K_EMPTY + s), 1);
-      mbar_init(bar(BR::V_FULL + s), 1);
-      mbar_init(bar(BR::V_EMPTY + s), 1);
+      mbar_init(bar(BR::RING_FULL + s), 1);
+      mbar_init(bar(BR::RING_EMPTY + s), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -222,191 +255,234 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int H = p.heads;
-
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t kv_it = 0, it = 0;
+      uint32_t r = 0, it = 0;  // ring sequence (K(g) = 2g, V(g) = 2g + 1), item count
       // Phase of the newest copy issued on each full barrier (-1: none yet), so
       // that an early stop can wait for copies still in flight.
-      int q_last = -1, k_last[S], v_last[S];
-      for (int s = 0; s < S; ++s) k_last[s] = v_last[s] = -1;
+      int q_last = -1, ring_last[S];
+      for (int s = 0; s < S; ++s) ring_last[s] = -1;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
         const Item w = decode_item(p, item);
         const AttnNode& nd = p.nodes[w.node];
         if (it > 0 && !wait_bar(bar(B_Q_EMPTY), (it - 1) & 1, ctl, 0x101)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(B_Q_FULL), C::kTileBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(sbase + C::kQOff + pn * C::kPanelBytes, &p.tm_q, pn * 64, w.head,
-                      nd.q_row0 + w.qtile * 128, bar(B_Q_FULL));
+        mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * C::kTileBytes);
+        for (int q = 0; q < 2; ++q)
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(sbase + C::kQOff + q * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
+                        pn * 64, w.head, nd.q_row0 + (2 * w.pair + q) * 128, bar(B_Q_FULL));
         q_last = it & 1;
-        for (int t = 0; t < nd.n_pages; ++t, ++kv_it) {
+        for (int t = 0; ok && t < nd.n_pages; ++t) {
           const uint32_t page = p.pages[nd.page0 + t] & kPageMask;
-          const int s = kv_it % S;
-          const uint32_t ph = (kv_it / S) & 1;
           const int32_t yk = (int32_t)(((int64_t)page * 2 * H + w.head) * 128);
-          const int32_t yv = yk + H * 128;
-          if (kv_it >= (uint32_t)S && !wait_bar(bar(BR::K_EMPTY + s), ph ^ 1, ctl, 0x102)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(BR::K_FULL + s), C::kTileBytes);
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_2d(sbase + C::kKOff + s * C::kTileBytes + pn * C::kPanelBytes, &p.tm_kv,
-                        pn * 64, yk, bar(BR::K_FULL + s));
-          k_last[s] = (int)ph;
-          if (kv_it >= (uint32_t)S && !wait_bar(bar(BR::V_EMPTY + s), ph ^ 1, ctl, 0x103)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(BR::V_FULL + s), C::kTileBytes);
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_2d(sbase + C::kVOff + s * C::kTileBytes + pn * C::kPanelBytes, &p.tm_kv,
-                        pn * 64, yv, bar(BR::V_FULL + s));
-          v_last[s] = (int)ph;
+          for (int kv = 0; kv < 2; ++kv, ++r) {
+            const int s = r % S;
+            const uint32_t ph = (r / S) & 1;
+            if (r >= (uint32_t)S && !wait_bar(bar(BR::RING_EMPTY + s), ph ^ 1, ctl, 0x102)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(BR::RING_FULL + s), C::kTileBytes);
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_2d(sbase + C::kRingOff + s * C::kTileBytes + pn * C::kPanelBytes, &p.tm_kv,
+                          pn * 64, yk + kv * H * 128, bar(BR::RING_FULL + s));
+            ring_last[s] = (int)ph;
+          }
         }
       }
       if (!ok) {
         // Stopping early: let the copies already issued land before the CTA's
         // shared memory is released.
         if (q_last >= 0) drain_wait(bar(B_Q_FULL), (uint32_t)q_last);
-        for (int s = 0; s < S; ++s) {
-          if (k_last[s] >= 0) drain_wait(bar(BR::K_FULL + s), (uint32_t)k_last[s]);
-          if (v_last[s] >= 0) drain_wait(bar(BR::V_FULL + s), (uint32_t)v_last[s]);
-        }
+        for (int s = 0; s < S; ++s)
+          if (ring_last[s] >= 0) drain_wait(bar(BR::RING_FULL + s), (uint32_t)ring_last[s]);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
-      uint32_t kv_it = 0, it = 0;
+      uint32_t g = 0, it = 0;  // global K/V tile count, item count
       bool ok = true;
-      auto issue_pv = [&](uint32_t g, bool first) -> bool {
-        const int s = g % S;
-        const uint32_t b = g & 1;
-        if (!wait_bar(bar(B_P_FULL + b), (g >> 1) & 1, ctl, 0x111)) return false;
-        if (!wait_bar(bar(BR::V_FULL + s), (g / S) & 1, ctl, 0x112)) return false;
-        if (first && it > 0 && !wait_bar(bar(B_O_EMPTY), (it - 1) & 1, ctl, 0x113)) return false;
-        tc_fence_after();
-        const uint32_t vaddr = sbase + C::kVOff + s * C::kTileBytes;
+      auto ring_wait = [&](uint32_t r, int code) -> bool {
+        return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
+      };
+      auto slot_addr = [&](uint32_t r) -> uint32_t {
+        return sbase + C::kRingOff + (r % S) * C::kTileBytes;
+      };
+      // S_w = Q_w K(t)^T into TMEM columns 128 w.
+      auto issue_s = [&](int w, uint32_t t) {
+        const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
+        const uint32_t kaddr = slot_addr(2 * t);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+          mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off), C::kIdescS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_w (+)= P_w V(t), P_w read from TMEM (bf16 in S_w's first 64 columns).
+      auto issue_pv = [&](int w, uint32_t t, bool accumulate) {
+        const uint32_t vaddr = slot_addr(2 * t + 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::kColO, tmem + C::kColP + b * 64 + kk * 8, desc_mn(vaddr + kk * 2048),
-                 C::kIdescO, (first && kk == 0) ? 0u : 1u);
-        tc_commit(bar(B_PV_DONE));
-        tc_commit(bar(BR::V_EMPTY + s));
-        return true;
+          mma_ts(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w + kk * 8,
+                 desc_mn(vaddr + kk * 2048), C::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
       };
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
         const Item w = decode_item(p, item);
-        const int n_pages = p.nodes[w.node].n_pages;
+        const int n = p.nodes[w.node].n_pages;
         if (!wait_bar(bar(B_Q_FULL), it & 1, ctl, 0x110)) { ok = false; break; }
+        if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
         tc_fence_after();
-        for (int t = 0; t < n_pages; ++t, ++kv_it) {
-          const int s = kv_it % S;
-          const uint32_t b = kv_it & 1;
-          if (!wait_bar(bar(BR::K_FULL + s), (kv_it / S) & 1, ctl, 0x114)) { ok = false; break; }
+        issue_s(0, g);
+        tc_commit(bar(B_S_FULL + 0));
+        issue_s(1, g);
+        tc_commit(bar(B_S_FULL + 1));
+        tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));
+        if (n == 1) tc_commit(bar(B_Q_EMPTY));
+        for (int j = 0; j < n; ++j, ++g) {
+          const bool more = j + 1 < n;
+          // ---- query tile 0: P0 V(g), then S0 for the next K/V tile
+          if (!wait_bar(bar(B_P_FULL + 0), g & 1, ctl, 0x112)) { ok = false; break; }
+          if (j == 0 && it > 0 && !wait_bar(bar(B_O_EMPTY + 0), (it - 1) & 1, ctl, 0x113)) { ok = false; break; }
+          if (!ring_wait(2 * g + 1, 0x114)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t qaddr = sbase + C::kQOff;
-          const uint32_t kaddr = sbase + C::kKOff + s * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-            mma_ss(tmem + C::kColS + b * 128, desc_k(qaddr + off), desc_k(kaddr + off), C::kIdescS,
-                   kk > 0 ? 1u : 0u);
+          issue_pv(0, g, j > 0);
+          if (more) {
+            if (!ring_wait(2 * g + 2, 0x115)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(0, g + 1);
+            tc_commit(bar(B_S_FULL + 0));
+          } else {
+            tc_commit(bar(B_O_FULL + 0));
           }
-          tc_commit(bar(B_S_FULL + b));
-          tc_commit(bar(BR::K_EMPTY + s));
-          if (t == n_pages - 1) tc_commit(bar(B_Q_EMPTY));
-          if (t > 0 && !issue_pv(kv_it - 1, t == 1)) { ok = false; break; }
+          // ---- query tile 1
+          if (!wait_bar(bar(B_P_FULL + 1), g & 1, ctl, 0x116)) { ok = false; break; }
+          if (j == 0 && it > 0 && !wait_bar(bar(B_O_EMPTY + 1), (it - 1) & 1, ctl, 0x117)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, g, j > 0);
+          tc_commit(bar(BR::RING_EMPTY + (2 * g + 1) % S));  // V(g) read by both tiles
+          if (more) {
+            issue_s(1, g + 1);
+            tc_commit(bar(B_S_FULL + 1));
+            tc_commit(bar(BR::RING_EMPTY + (2 * g + 2) % S));  // K(g+1) read by both tiles
+            if (j + 2 == n) tc_commit(bar(B_Q_EMPTY));
+          } else {
+            tc_commit(bar(B_O_FULL + 1));
+          }
         }
-        if (!ok) break;
-        if (!issue_pv(kv_it - 1, n_pages == 1)) { ok = false; break; }
-        tc_commit(bar(B_O_FULL));
       }
       // Wait (bounded) until every MMA issued by this thread has finished.
       tc_commit(bar(B_DRAIN));
       drain_wait(bar(B_DRAIN), 0);
     }
+  }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    regs_inc<kRegsHigh>();
+    const int wq = (warp - 4) >> 2;  // query tile of this warpgroup
+    const int quarter = warp & 3;    // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tS = trow + C::kColS + 128 * wq;
+    const uint32_t tO = trow + C::kColO + 128 * wq;
     const float sl2 = p.scale_log2;
-    uint32_t kv_it = 0, it = 0;
+    uint32_t g = 0, it = 0;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
       const Item w = decode_item(p, item);
       const AttnNode& nd = p.nodes[w.node];
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
-      for (int t = 0; t < nd.n_pages; ++t, ++kv_it) {
-        const uint32_t b = kv_it & 1;
-        ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + b), (kv_it >> 1) & 1, ctl, 0x120));
+      for (int t = 0; t < nd.n_pages; ++t, ++g) {
+        ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
         tc_fence_after();
         const int valid = (int)(p.pages[nd.page0 + t] >> 25) + 1;
+        // The whole S row in one TMEM round trip.
         float sv[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          tmem_ld32(trow + C::kColS + b * 128 + c * 32,
-                    *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
         tmem_wait_ld();
-        float mx = -INFINITY;
+        if (valid < 128) {  // partial last page of an entry: drop the padding keys
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          sv[i] = i < valid ? sv[i] : -INFINITY;
-          mx = fmaxf(mx, sv[i]);
+          for (int i = 0; i < 128; ++i) sv[i] = i < valid ? sv[i] : -INFINITY;
         }
-        const float m_new = fmaxf(m_run, mx * sl2);
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(sv[i], sv[8 + i], sv[16 + i]);
+#pragma unroll
+        for (int k = 24; k < 120; k += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], sv[k + i], sv[k + 8 + i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], sv[120 + i]);
+        const float mrow = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
+        const float m_new = fmaxf(m_run, mrow * sl2);
         const bool grow = __any_sync(0xffffffffu, t > 0 && m_new > m_run + 8.f);
         if (t == 0) {
           m_run = m_new;
         } else if (grow) {
-          // Bring O up to the new max: wait for the previous P.V, scale O in TMEM.
-          ok = __all_sync(0xffffffffu, wait_bar(bar(B_PV_DONE), (kv_it - 1) & 1, ctl, 0x121));
-          if (!ok) break;
-          tc_fence_after();
+          // Bring O up to the new max. The P.V of the previous tile is done:
+          // it was issued before this tile's S, whose completion we waited for.
           const float alpha = ex2_approx(m_run - m_new);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(trow + C::kColO + c * 32, o);
+            tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(trow + C::kColO + c * 32, o);
+            tmem_st32(tO + c * 32, o);
           }
-          tmem_wait_st();
           l_run *= alpha;
           m_run = m_new;
         }
-        float sum = 0.f;
+        // P = 2^(S log2e/sqrt(d) - m), packed to bf16 into S's first 64 columns.
+        const float negm = -m_run;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < 8; ++c) {  // 16 columns of S -> 8 columns of P
+          uint32_t pk[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(fmaf(sv[c * 32 + 2 * i], sl2, -m_run));
-            const float p1 = ex2_approx(fmaf(sv[c * 32 + 2 * i + 1], sl2, -m_run));
-            sum += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 8; ++i) {
+            const float x0 = fmaf(sv[c * 16 + 2 * i], sl2, negm);
+            const float x1 = fmaf(sv[c * 16 + 2 * i + 1], sl2, negm);
+            float y0, y1;
+            if (((c & 1) * 16 + 2 * i) < kEmuPerChunk) {
+              exp2_poly2(x0, x1, y0, y1);
+            } else {
+              y0 = ex2_approx(x0);
+              y1 = ex2_approx(x1);
+            }
+            acc[i & 3] += y0 + y1;
+            pk[i] = pack_bf16x2(y0, y1);
           }
-          tmem_st16(trow + C::kColP + b * 64 + c * 16, pk);
+          tmem_st8(tS + c * 8, pk);
         }
-        l_run += sum;
+        l_run += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + b));
+        mbar_arrive(bar(B_P_FULL + wq));
       }
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, wait_bar(bar(B_O_FULL), it & 1, ctl, 0x122));
+      ok = __all_sync(0xffffffffu, wait_bar(bar(B_O_FULL + wq), it & 1, ctl, 0x122 + wq));
       if (!ok) break;
       tc_fence_after();
       const float inv = 1.f / l_run;
-      const int q_local = w.qtile * 128 + row;
+      const int q_local = (2 * w.pair + wq) * 128 + row;
       const bool store = q_local < p.q_rows;
       uint4* orow = reinterpret_cast<uint4*>(
           p.out + ((int64_t)(nd.q_row0 + q_local) * H + w.head) * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(trow + C::kColO + c * 32, o);
+        tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -419,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(B_O_EMPTY));
+      mbar_arrive(bar(B_O_EMPTY + wq));
     }
   }
 
@@ -450,12 +526,21 @@ template <int D>
 int launch(const AttnParams& prm, int grid, cudaStream_t stream) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
+  static int num_regs = 0;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(round_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     Cfg<D>::kSmemBytes);
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, round_attn_kernel<D>);
+    if (attr_err == cudaSuccess) num_regs = fa.numRegs;
   });
   if (attr_err != cudaSuccess)
     return fail(WAVE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  // setmaxnreg.inc waits until registers are free: with fewer registers per
+  // thread at launch than the split assumes it would never return.
+  if ((uint32_t)num_regs < kRegsLaunch)
+    return fail(WAVE_ERR_UNSUPPORTED, "round_attn_kernel compiled with %d registers per thread; "
+                "its warpgroup register split needs %u", num_regs, kRegsLaunch);
   round_attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "round_attn_kernel launch: %s", cudaGetErrorString(e));
@@ -519,6 +604,7 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
     return offs[a + 1] - offs[a] > offs[b + 1] - offs[b];
   });
   const int n_qtiles = (T + 127) / 128;
+  const int n_pairs = (n_qtiles + 1) / 2;
   int32_t item0 = 0, w = 0;
   for (int k = 0; k < n_active; ++k) {
     const int i = order[k];
@@ -527,10 +613,10 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
     nd.page0 = w;
     nd.n_pages = offs[i + 1] - offs[i];
     nd.item0 = item0;
-    nd.n_qtiles = n_qtiles;
+    nd.n_pairs = n_pairs;
     for (int32_t rr = offs[i]; rr < offs[i + 1]; ++rr)
       prm.pages[w++] = (uint32_t)rows[2 * rr] | ((uint32_t)(rows[2 * rr + 1] - 1) << 25);
-    item0 += H * n_qtiles;
+    item0 += H * n_pairs;
   }
   prm.n_items = item0;
   const int grid = std::min(prm.n_items, kv->num_sms);
