@@ -76,11 +76,16 @@ _SIGS = {
 }
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libwave.so (once). Raises if it has not been built."""
+def load(path: str = None) -> ctypes.CDLL:
+    """Load libwave.so (once). Raises if it has not been built.
+
+    The library next to this file is used unless ``path`` or the environment
+    variable WAVE_LIBRARY names another build of it.
+    """
     global _lib
     if _lib is not None:
         return _lib
+    path = path or os.environ.get("WAVE_LIBRARY") or LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m block_causal_attention_wave_b200.build`")

@@ -31,13 +31,15 @@ def sources():
     return sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cpp")))
 
 
-def build(verbose_ptxas: bool = False, out: str = LIB) -> str:
-    objdir = os.path.join(PKG, "_build")
+def build(verbose_ptxas: bool = False, out: str = LIB, defines=()) -> str:
+    """Compile every source into ``out``; ``defines`` are extra -D macros."""
+    objdir = os.path.join(PKG, "_build", os.path.splitext(os.path.basename(out))[0])
     os.makedirs(objdir, exist_ok=True)
     common = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-Wall",
                      "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc")]
     if verbose_ptxas:
         common += ["-Xptxas", "-v"]
+    common += [f"-D{d}" for d in defines]
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")

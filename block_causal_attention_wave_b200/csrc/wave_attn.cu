@@ -63,14 +63,15 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "regis
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
 constexpr uint32_t kPageMask = (1u << 25) - 1;  // page id bits of a page word
+constexpr int64_t kCounterOffset = 128;         // work-queue counter in the pool header
 
 struct AttnNode {
   int32_t q_row0;    // first row of this node in Q / O
   int32_t page0;     // first page word
   int32_t n_pages;   // key pages
   int32_t item0;     // first work item
-  int32_t n_pairs;   // ceil(ceil(T / 128) / 2): pairs of 128-row query tiles
-  int32_t pad;
+  int32_t n_pairs;   // ceil(n_qtiles / 2): pairs of 128-row query tiles
+  int32_t n_qtiles;  // ceil(T / 128)
 };
 
 struct AttnParams {
@@ -78,6 +79,7 @@ struct AttnParams {
   CUtensorMap tm_kv;  // pool page region as rows of d
   uint16_t* out;      // O, bf16 [rows][H][d]
   int32_t* status;    // device status word (pool header)
+  int32_t* counter;   // work-queue counter, zero at launch (pool header)
   float scale_log2;   // log2(e) / sqrt(d)
   int32_t heads;
   int32_t n_nodes;
@@ -90,8 +92,16 @@ struct AttnParams {
 static_assert(sizeof(AttnParams) <= 32760, "kernel parameter space is 32 KB");
 
 // Softmax columns (of each 32) whose exp2 runs on the FMA pipe (polynomial)
-// instead of the special-function unit.
-constexpr int kEmuPerChunk = 8;
+// instead of the special-function unit; even, 0..32.
+#ifndef WAVE_EMU_PER_CHUNK
+#define WAVE_EMU_PER_CHUNK 8
+#endif
+constexpr int kEmuPerChunk = WAVE_EMU_PER_CHUNK;
+// 1: scale/shift of S and the row sum use packed fp32x2 FMA/ADD.
+#ifndef WAVE_PACKED_FMA
+#define WAVE_PACKED_FMA 1
+#endif
+static_assert(kEmuPerChunk % 2 == 0 && kEmuPerChunk >= 0 && kEmuPerChunk <= 32, "emulated share");
 
 template <int D>
 struct Cfg {
@@ -122,15 +132,18 @@ enum : int {
   B_O_FULL = B_P_FULL + 2,  // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2, // 2: epilogue has read O_w (128 arrivals)
   B_DRAIN = B_O_EMPTY + 2,
-  B_RING_FULL,              // kSlots each from here
+  B_ITEM_FULL,              // 2: next work item published by the producer
+  B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by the MMA thread and 8 softmax warps
+  B_RING_FULL = B_ITEM_EMPTY + 2,  // kSlots each from here
 };
+constexpr int kItemSlots = 2;
 
 template <int D>
 struct Bars {
   static constexpr int kS = Cfg<D>::kSlots;
   static constexpr int RING_FULL = B_RING_FULL, RING_EMPTY = RING_FULL + kS,
                        COUNT = RING_EMPTY + kS;
-  static_assert(COUNT * 8 + 16 <= 512, "barrier area");
+  static_assert(COUNT * 8 + 16 + 4 * kItemSlots <= 512, "barrier area");
 };
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
@@ -175,6 +188,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 
 struct Item {
   int node, head, pair;
+  bool two;  // the pair's second query tile holds rows of the node
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
@@ -182,7 +196,8 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   while (n + 1 < p.n_nodes && item >= p.nodes[n + 1].item0) ++n;
   const int j = item - p.nodes[n].item0;
   const int np = p.nodes[n].n_pairs;
-  return Item{n, j / np, j % np};
+  const int pair = j % np;
+  return Item{n, j / np, pair, 2 * pair + 1 < p.nodes[n].n_qtiles};
 }
 
 // 2^x for a pair of x <= 8 on the FMA pipe: x = j + f, j = round(x),
@@ -222,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * BR::COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 4);
+  volatile int* item_q = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 8);
   const Ctl ctl{abort_flag, p.status};
 
   const int warp = threadIdx.x >> 5;
@@ -235,6 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_P_FULL + w), 128);
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
+    }
+    for (int k = 0; k < kItemSlots; ++k) {
+      mbar_init(bar(B_ITEM_FULL + k), 1);
+      mbar_init(bar(B_ITEM_EMPTY + k), 1 + 8);  // MMA thread + one lane per softmax warp
     }
     mbar_init(bar(B_DRAIN), 1);
     for (int s = 0; s < S; ++s) {
@@ -255,132 +275,161 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int H = p.heads;
+
+  // Work items, longest key list first, are handed out dynamically: the
+  // producer claims the next one (the CTA's first is blockIdx.x, later ones
+  // come from a global counter) and publishes it to the other roles through a
+  // two-slot queue in shared memory. An id >= n_items tells every role to stop.
+  auto next_item = [&](uint32_t k, int code, int& item) -> bool {  // consumer side
+    if (!wait_bar(bar(B_ITEM_FULL + (k % kItemSlots)), (k / kItemSlots) & 1, ctl, code))
+      return false;
+    item = item_q[k % kItemSlots];
+    return true;
+  };
+
   if (warp < 4) {
-  regs_dec<kRegsLow>();
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t r = 0, it = 0;  // ring sequence (K(g) = 2g, V(g) = 2g + 1), item count
-      // Phase of the newest copy issued on each full barrier (-1: none yet), so
-      // that an early stop can wait for copies still in flight.
-      int q_last = -1, ring_last[S];
-      for (int s = 0; s < S; ++s) ring_last[s] = -1;
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-        const Item w = decode_item(p, item);
-        const AttnNode& nd = p.nodes[w.node];
-        if (it > 0 && !wait_bar(bar(B_Q_EMPTY), (it - 1) & 1, ctl, 0x101)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * C::kTileBytes);
-        for (int q = 0; q < 2; ++q)
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(sbase + C::kQOff + q * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
-                        pn * 64, w.head, nd.q_row0 + (2 * w.pair + q) * 128, bar(B_Q_FULL));
-        q_last = it & 1;
-        for (int t = 0; ok && t < nd.n_pages; ++t) {
-          const uint32_t page = p.pages[nd.page0 + t] & kPageMask;
-          const int32_t yk = (int32_t)(((int64_t)page * 2 * H + w.head) * 128);
-          for (int kv = 0; kv < 2; ++kv, ++r) {
-            const int s = r % S;
-            const uint32_t ph = (r / S) & 1;
-            if (r >= (uint32_t)S && !wait_bar(bar(BR::RING_EMPTY + s), ph ^ 1, ctl, 0x102)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(bar(BR::RING_FULL + s), C::kTileBytes);
+    regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        uint32_t r = 0, it = 0;  // ring sequence (K(g) = 2g, V(g) = 2g + 1), item count
+        // Phase of the newest copy issued on each full barrier (-1: none yet),
+        // so that an early stop can wait for copies still in flight.
+        int q_last = -1, ring_last[S];
+        for (int s = 0; s < S; ++s) ring_last[s] = -1;
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+          const int slot = k % kItemSlots;
+          if (k >= (uint32_t)kItemSlots &&
+              !wait_bar(bar(B_ITEM_EMPTY + slot), ((k / kItemSlots) & 1) ^ 1, ctl, 0x100)) {
+            ok = false;
+            break;
+          }
+          const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
+          item_q[slot] = item;
+          mbar_arrive(bar(B_ITEM_FULL + slot));
+          if (item >= p.n_items) break;
+          const Item w = decode_item(p, item);
+          const AttnNode& nd = p.nodes[w.node];
+          if (it > 0 && !wait_bar(bar(B_Q_EMPTY), (it - 1) & 1, ctl, 0x101)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(B_Q_FULL), (w.two ? 2 : 1) * C::kTileBytes);
+          for (int q = 0; q < (w.two ? 2 : 1); ++q)
             for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_2d(sbase + C::kRingOff + s * C::kTileBytes + pn * C::kPanelBytes, &p.tm_kv,
-                          pn * 64, yk + kv * H * 128, bar(BR::RING_FULL + s));
-            ring_last[s] = (int)ph;
+              tma_load_3d(sbase + C::kQOff + q * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
+                          pn * 64, w.head, nd.q_row0 + (2 * w.pair + q) * 128, bar(B_Q_FULL));
+          q_last = it & 1;
+          ++it;
+          for (int t = 0; ok && t < nd.n_pages; ++t) {
+            const uint32_t page = p.pages[nd.page0 + t] & kPageMask;
+            const int32_t yk = (int32_t)(((int64_t)page * 2 * H + w.head) * 128);
+            for (int kv = 0; kv < 2; ++kv, ++r) {
+              const int s = r % S;
+              const uint32_t ph = (r / S) & 1;
+              if (r >= (uint32_t)S && !wait_bar(bar(BR::RING_EMPTY + s), ph ^ 1, ctl, 0x102)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(bar(BR::RING_FULL + s), C::kTileBytes);
+              for (int pn = 0; pn < C::kPanels; ++pn)
+                tma_load_2d(sbase + C::kRingOff + s * C::kTileBytes + pn * C::kPanelBytes,
+                            &p.tm_kv, pn * 64, yk + kv * H * 128, bar(BR::RING_FULL + s));
+              ring_last[s] = (int)ph;
+            }
           }
         }
+        if (!ok) {
+          // Stopping early: let the copies already issued land before the
+          // CTA's shared memory is released.
+          if (q_last >= 0) drain_wait(bar(B_Q_FULL), (uint32_t)q_last);
+          for (int s = 0; s < S; ++s)
+            if (ring_last[s] >= 0) drain_wait(bar(BR::RING_FULL + s), (uint32_t)ring_last[s]);
+        }
       }
-      if (!ok) {
-        // Stopping early: let the copies already issued land before the CTA's
-        // shared memory is released.
-        if (q_last >= 0) drain_wait(bar(B_Q_FULL), (uint32_t)q_last);
-        for (int s = 0; s < S; ++s)
-          if (ring_last[s] >= 0) drain_wait(bar(BR::RING_FULL + s), (uint32_t)ring_last[s]);
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- tcgen05 issuer
+      if (lane == 0) {
+        // g: K/V tiles consumed; gw/itw: tiles/items processed by query tile w.
+        uint32_t g = 0, it = 0, gw[2] = {0, 0}, itw[2] = {0, 0};
+        bool ok = true;
+        auto ring_wait = [&](uint32_t r, int code) -> bool {
+          return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
+        };
+        auto slot_addr = [&](uint32_t r) -> uint32_t {
+          return sbase + C::kRingOff + (r % S) * C::kTileBytes;
+        };
+        // S_w = Q_w K(t)^T into TMEM columns 128 w.
+        auto issue_s = [&](int w, uint32_t t) {
+          const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
+          const uint32_t kaddr = slot_addr(2 * t);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+            mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off),
+                   C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+        };
+        // O_w (+)= P_w V(t), P_w read from TMEM (bf16 in S_w's first 64 columns).
+        auto issue_pv = [&](int w, uint32_t t, bool accumulate) {
+          const uint32_t vaddr = slot_addr(2 * t + 1);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w + kk * 8,
+                   desc_mn(vaddr + kk * 2048), C::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
+        };
+        for (uint32_t k = 0; ok; ++k) {
+          int item;
+          if (!next_item(k, 0x118, item)) { ok = false; break; }
+          mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
+          if (item >= p.n_items) break;
+          const Item w = decode_item(p, item);
+          const int n = p.nodes[w.node].n_pages;
+          const int nq = w.two ? 2 : 1;
+          if (!wait_bar(bar(B_Q_FULL), it & 1, ctl, 0x110)) { ok = false; break; }
+          if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
+          tc_fence_after();
+          for (int q = 0; q < nq; ++q) {
+            issue_s(q, g);
+            tc_commit(bar(B_S_FULL + q));
+          }
+          tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));
+          if (n == 1) tc_commit(bar(B_Q_EMPTY));
+          for (int j = 0; j < n; ++j, ++g) {
+            const bool more = j + 1 < n;
+            for (int q = 0; q < nq; ++q) {
+              if (!wait_bar(bar(B_P_FULL + q), gw[q] & 1, ctl, 0x112 + q)) { ok = false; break; }
+              if (j == 0 && itw[q] > 0 &&
+                  !wait_bar(bar(B_O_EMPTY + q), (itw[q] - 1) & 1, ctl, 0x114 + q)) {
+                ok = false;
+                break;
+              }
+              if (q == 0 && !ring_wait(2 * g + 1, 0x116)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(q, g, j > 0);
+              ++gw[q];
+              if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * g + 1) % S));  // V(g) done
+              if (more) {
+                if (q == 0 && !ring_wait(2 * g + 2, 0x117)) { ok = false; break; }
+                tc_fence_after();
+                issue_s(q, g + 1);
+                tc_commit(bar(B_S_FULL + q));
+                if (q == nq - 1) {
+                  tc_commit(bar(BR::RING_EMPTY + (2 * g + 2) % S));  // K(g+1) done
+                  if (j + 2 == n) tc_commit(bar(B_Q_EMPTY));
+                }
+              } else {
+                tc_commit(bar(B_O_FULL + q));
+              }
+            }
+            if (!ok) break;
+          }
+          for (int q = 0; q < nq; ++q) ++itw[q];
+          ++it;
+        }
+        // Wait (bounded) until every MMA issued by this thread has finished.
+        tc_commit(bar(B_DRAIN));
+        drain_wait(bar(B_DRAIN), 0);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ tcgen05 issuer
-    if (lane == 0) {
-      uint32_t g = 0, it = 0;  // global K/V tile count, item count
-      bool ok = true;
-      auto ring_wait = [&](uint32_t r, int code) -> bool {
-        return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
-      };
-      auto slot_addr = [&](uint32_t r) -> uint32_t {
-        return sbase + C::kRingOff + (r % S) * C::kTileBytes;
-      };
-      // S_w = Q_w K(t)^T into TMEM columns 128 w.
-      auto issue_s = [&](int w, uint32_t t) {
-        const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
-        const uint32_t kaddr = slot_addr(2 * t);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-          mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off), C::kIdescS,
-                 kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_w (+)= P_w V(t), P_w read from TMEM (bf16 in S_w's first 64 columns).
-      auto issue_pv = [&](int w, uint32_t t, bool accumulate) {
-        const uint32_t vaddr = slot_addr(2 * t + 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w + kk * 8,
-                 desc_mn(vaddr + kk * 2048), C::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
-      };
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-        const Item w = decode_item(p, item);
-        const int n = p.nodes[w.node].n_pages;
-        if (!wait_bar(bar(B_Q_FULL), it & 1, ctl, 0x110)) { ok = false; break; }
-        if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
-        tc_fence_after();
-        issue_s(0, g);
-        tc_commit(bar(B_S_FULL + 0));
-        issue_s(1, g);
-        tc_commit(bar(B_S_FULL + 1));
-        tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));
-        if (n == 1) tc_commit(bar(B_Q_EMPTY));
-        for (int j = 0; j < n; ++j, ++g) {
-          const bool more = j + 1 < n;
-          // ---- query tile 0: P0 V(g), then S0 for the next K/V tile
-          if (!wait_bar(bar(B_P_FULL + 0), g & 1, ctl, 0x112)) { ok = false; break; }
-          if (j == 0 && it > 0 && !wait_bar(bar(B_O_EMPTY + 0), (it - 1) & 1, ctl, 0x113)) { ok = false; break; }
-          if (!ring_wait(2 * g + 1, 0x114)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(0, g, j > 0);
-          if (more) {
-            if (!ring_wait(2 * g + 2, 0x115)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(0, g + 1);
-            tc_commit(bar(B_S_FULL + 0));
-          } else {
-            tc_commit(bar(B_O_FULL + 0));
-          }
-          // ---- query tile 1
-          if (!wait_bar(bar(B_P_FULL + 1), g & 1, ctl, 0x116)) { ok = false; break; }
-          if (j == 0 && it > 0 && !wait_bar(bar(B_O_EMPTY + 1), (it - 1) & 1, ctl, 0x117)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(1, g, j > 0);
-          tc_commit(bar(BR::RING_EMPTY + (2 * g + 1) % S));  // V(g) read by both tiles
-          if (more) {
-            issue_s(1, g + 1);
-            tc_commit(bar(B_S_FULL + 1));
-            tc_commit(bar(BR::RING_EMPTY + (2 * g + 2) % S));  // K(g+1) read by both tiles
-            if (j + 2 == n) tc_commit(bar(B_Q_EMPTY));
-          } else {
-            tc_commit(bar(B_O_FULL + 1));
-          }
-        }
-      }
-      // Wait (bounded) until every MMA issued by this thread has finished.
-      tc_commit(bar(B_DRAIN));
-      drain_wait(bar(B_DRAIN), 0);
-    }
-  }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     regs_inc<kRegsHigh>();
@@ -391,12 +440,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = trow + C::kColS + 128 * wq;
     const uint32_t tO = trow + C::kColO + 128 * wq;
     const float sl2 = p.scale_log2;
-    uint32_t g = 0, it = 0;
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
+    uint32_t g = 0, it = 0;  // tiles and items processed by this warpgroup
+    for (uint32_t k = 0;; ++k) {
+      int item;
+      bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, item));
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
+      if (item >= p.n_items) break;
       const Item w = decode_item(p, item);
+      if (wq == 1 && !w.two) continue;  // the pair's second tile lies past the node
       const AttnNode& nd = p.nodes[w.node];
       float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
       for (int t = 0; t < nd.n_pages; ++t, ++g) {
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
@@ -445,14 +500,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P = 2^(S log2e/sqrt(d) - m), packed to bf16 into S's first 64 columns.
         const float negm = -m_run;
+#if WAVE_PACKED_FMA
+        const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(negm, negm);
+        uint64_t acc2[2] = {0, 0};
+#else
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#endif
 #pragma unroll
         for (int c = 0; c < 8; ++c) {  // 16 columns of S -> 8 columns of P
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float x0 = fmaf(sv[c * 16 + 2 * i], sl2, negm);
-            const float x1 = fmaf(sv[c * 16 + 2 * i + 1], sl2, negm);
+            float x0, x1;
+#if WAVE_PACKED_FMA
+            f2_unpack(f2_fma(f2_pack(sv[c * 16 + 2 * i], sv[c * 16 + 2 * i + 1]), scale2, negm2), x0,
+                      x1);
+#else
+            x0 = fmaf(sv[c * 16 + 2 * i], sl2, negm);
+            x1 = fmaf(sv[c * 16 + 2 * i + 1], sl2, negm);
+#endif
             float y0, y1;
             if (((c & 1) * 16 + 2 * i) < kEmuPerChunk) {
               exp2_poly2(x0, x1, y0, y1);
@@ -460,11 +526,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               y0 = ex2_approx(x0);
               y1 = ex2_approx(x1);
             }
+#if WAVE_PACKED_FMA
+            acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(y0, y1));
+#else
             acc[i & 3] += y0 + y1;
+#endif
             pk[i] = pack_bf16x2(y0, y1);
           }
           tmem_st8(tS + c * 8, pk);
         }
+#if WAVE_PACKED_FMA
+        float acc[4];
+        f2_unpack(acc2[0], acc[0], acc[1]);
+        f2_unpack(acc2[1], acc[2], acc[3]);
+#endif
         l_run += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();
@@ -496,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(bar(B_O_EMPTY + wq));
+      ++it;
     }
   }
 
@@ -591,6 +667,7 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
   prm.tm_kv = kv->tm_kv;
   prm.out = static_cast<uint16_t*>(O);
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
+  prm.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
   prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   prm.heads = H;
   prm.q_rows = T;
@@ -614,6 +691,7 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
     nd.n_pages = offs[i + 1] - offs[i];
     nd.item0 = item0;
     nd.n_pairs = n_pairs;
+    nd.n_qtiles = n_qtiles;
     for (int32_t rr = offs[i]; rr < offs[i + 1]; ++rr)
       prm.pages[w++] = (uint32_t)rows[2 * rr] | ((uint32_t)(rows[2 * rr + 1] - 1) << 25);
     item0 += H * n_pairs;
@@ -621,5 +699,7 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
   prm.n_items = item0;
   const int grid = std::min(prm.n_items, kv->num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(prm.counter, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "cudaMemsetAsync(work counter): %s", cudaGetErrorString(e));
   return D == 128 ? launch<128>(prm, grid, s) : launch<64>(prm, grid, s);
 }
