@@ -62,6 +62,10 @@ _SIGS = {
     "wave_round_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
                                        ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p]),
+    "wave_round_attn_static_scratch": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node),
+                                                      ctypes.c_int32, ctypes.c_int32,
+                                                      ctypes.c_void_p, ctypes.c_void_p,
+                                                      ctypes.c_void_p]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "wave_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.POINTER(Node), ctypes.c_int32,
@@ -240,6 +244,15 @@ class KVCache:
         _check(self.lib.wave_round_attn(self.h, nodes, len(active), _policy(policy),
                                         ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(O.data_ptr()),
                                         _stream_handle(stream)))
+        return O
+
+    def round_attn_static_scratch(self, active, policy, Q, O, stream=None):
+        """round_attn whose work-queue counter lives in the library's static
+        device array instead of the pool header (no per-call scratch)."""
+        nodes = _nodes(active)
+        _check(self.lib.wave_round_attn_static_scratch(
+            self.h, nodes, len(active), _policy(policy), ctypes.c_void_p(Q.data_ptr()),
+            ctypes.c_void_p(O.data_ptr()), _stream_handle(stream)))
         return O
 
     def status(self, stream=None):

@@ -629,9 +629,13 @@ int launch(const AttnParams& prm, int grid, cudaStream_t stream) {
 
 using namespace wavei;
 
-extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active,
-                               int32_t policy, const void* Q, void* O, void* stream) {
-  clear_error();
+namespace wavei {
+namespace {
+
+// One round of attention with the work-queue counter at `counter` (a device
+// int32 that this call sets to zero on `stream` before the launch).
+int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
+                    const void* Q, void* O, void* stream, int32_t* counter) {
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
   if (!valid_policy(policy)) return fail(WAVE_ERR_ARG, "unknown policy %d", policy);
@@ -667,7 +671,7 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
   prm.tm_kv = kv->tm_kv;
   prm.out = static_cast<uint16_t*>(O);
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
-  prm.counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
+  prm.counter = counter;
   prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   prm.heads = H;
   prm.q_rows = T;
@@ -702,4 +706,75 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
   cudaError_t e = cudaMemsetAsync(prm.counter, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "cudaMemsetAsync(work counter): %s", cudaGetErrorString(e));
   return D == 128 ? launch<128>(prm, grid, s) : launch<64>(prm, grid, s);
+}
+
+}  // namespace
+}  // namespace wavei
+
+extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active,
+                               int32_t policy, const void* Q, void* O, void* stream) {
+  clear_error();
+  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+  if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
+  int32_t* counter =
+      reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
+  return round_attn_impl(kv, active, n_active, policy, Q, O, stream, counter);
+}
+
+// ----------------------------------------------------------------------------
+// Static-scratch variant of wave_round_attn.
+//
+// wave_round_attn keeps its one piece of per-call device scratch -- the
+// work-queue counter that the persistent CTAs draw work items from -- in the
+// header of the caller's pool. This variant keeps it in the array below
+// instead, a file-scope device array of a fixed 256 bytes that exists on every
+// GPU that loads the library, until the process exits. Nothing is allocated
+// per call. Host code must not hand the array's name to a kernel (on the host
+// it is only a stand-in, not a device address); its device address is looked
+// up once per device with cudaGetSymbolAddress on the first call made with
+// that device current, and cached.
+namespace wavei {
+namespace {
+constexpr int kStaticScratchWords = 64;    // 256 bytes per device
+constexpr int kStaticScratchNeeded = 1;    // words used: the work-queue counter
+constexpr int kMaxDevices = 64;
+static_assert(kStaticScratchNeeded <= kStaticScratchWords, "static scratch too small");
+std::mutex g_scratch_mu;
+int32_t* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+}  // namespace wavei
+
+static __device__ __align__(256) int32_t g_round_attn_scratch[wavei::kStaticScratchWords];
+
+extern "C" int wave_round_attn_static_scratch(wave_kv* kv, const wave_node* active,
+                                              int32_t n_active, int32_t policy, const void* Q,
+                                              void* O, void* stream) {
+  clear_error();
+  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+  if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev != kv->device)
+    return fail(WAVE_ERR_ARG, "current device %d is not the pool's device %d", dev, kv->device);
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(WAVE_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices - 1);
+  // The scratch need does not grow with the round (one counter), so the only
+  // size limits are those wave_round_attn enforces: at most WAVE_MAX_NODES
+  // nodes and WAVE_MAX_PAGES_PER_ROUND key pages (WAVE_ERR_CAPACITY beyond).
+  int32_t* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_round_attn_scratch);
+      if (e != cudaSuccess || !ptr)
+        return fail(WAVE_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s",
+                    cudaGetErrorString(e));
+      g_scratch_addr[dev] = static_cast<int32_t*>(ptr);
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  // round_attn_impl zeroes the counter (word 0) on `stream` before launching.
+  return round_attn_impl(kv, active, n_active, policy, Q, O, stream, scratch);
 }

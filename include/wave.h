@@ -150,6 +150,27 @@ int wave_gather_table(const wave_kv* kv, const wave_node* active, int32_t n_acti
 int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
                     const void* Q, void* O, void* stream);
 
+/* wave_round_attn without per-call scratch from the caller. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory for the library while they run -- e.g. code inside CUDA stream
+ * capture, where cudaMalloc is refused, or a host whose device memory is all
+ * owned by another allocator. wave_round_attn keeps its per-call scratch (the
+ * 4-byte work-queue counter its persistent kernel draws work from) in the
+ * header of the caller's pool; this call keeps it in a 256-byte array that
+ * the library holds in device memory on every GPU it is loaded on, until the
+ * process exits. Arguments, results, layouts, limits (WAVE_MAX_NODES nodes,
+ * WAVE_MAX_PAGES_PER_ROUND key pages, WAVE_ERR_CAPACITY beyond) and error
+ * codes are those of wave_round_attn; timeouts are still reported by
+ * wave_kv_status. It allocates nothing: no cudaMalloc/cudaFree, no library
+ * allocator. The first call on a device, made with that device current (it
+ * must be the pool's device), looks up the array's device address once and
+ * caches it; make that first call before any stream capture. Each call zeroes
+ * the counter on `stream` before its launch. All calls on a device share the
+ * one array: calls whose kernels overlap on the GPU (e.g. on two streams
+ * without ordering) race on it and give undefined results. */
+int wave_round_attn_static_scratch(wave_kv* kv, const wave_node* active, int32_t n_active,
+                                   int32_t policy, const void* Q, void* O, void* stream);
+
 /* Synchronise `stream`, then read and clear the pool's device status word.
  * Returns WAVE_OK, WAVE_ERR_TIMEOUT if a kernel gave up on a bounded wait
  * (its output is then undefined), or WAVE_ERR_CUDA. */

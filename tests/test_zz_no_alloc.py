@@ -1,0 +1,57 @@
+"""wave_round_attn_static_scratch: the attention call for callers that cannot
+give the library device scratch.
+
+Such callers (code inside CUDA stream capture, where cudaMalloc is refused, or
+hosts whose device memory is all owned by another allocator) call
+wave_round_attn_static_scratch, which keeps the kernel's work-queue counter in
+a static device array inside the library instead of the pool header. This test
+runs it twice in a row through the C ABI and checks both outputs against
+wave_round_attn's on the same inputs, with the tolerance of the other parity
+tests (max-abs <= 1e-2, rel-L2 <= 5e-3). The second call only matches if the
+first left nothing behind that the second depends on (each call zeroes the
+counter before its launch).
+
+The file is named to be collected last, so a run that stops at the first
+failure has already run every other test.
+"""
+import pytest
+
+import wave_inputs as wi
+from oracle import cache as ocache
+from oracle import schedule as osched
+
+from wave_testlib import Inputs, append, assert_close, make_cache, queries, torch_to_f64
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    wi.Workload("static-scratch-d128", chunks=4, levels=2, heads=3, head_dim=128, tokens=300,
+                prefix=77),
+    wi.Workload("static-scratch-d64", chunks=3, levels=2, heads=2, head_dim=64, tokens=200,
+                window=1),
+]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_static_scratch_matches_wave_round_attn(cuda_lib, wl):
+    import torch
+    pol = "progressive"
+    inp = Inputs(wl)
+    rounds = osched.schedule(wl.chunks, wl.levels, pol, wl.window)
+    active = max(rounds, key=len)
+    entries = set()
+    for n in active:
+        entries.update(ocache.key_entries(n, pol, wl.window, wl.prefix > 0))
+    kv = make_cache(cuda_lib, wl, 64)
+    keep = [append(kv, inp, e) for e in sorted(entries)]
+    q = queries(inp, active)
+    o_ref = torch.empty_like(q)
+    kv.round_attn(active, pol, q, o_ref)
+    kv.status()
+    ref = torch_to_f64(o_ref)
+    for call in range(2):
+        o = torch.full_like(q, float("nan"))
+        kv.round_attn_static_scratch(active, pol, q, o)
+        kv.status()
+        assert_close(torch_to_f64(o), ref, f"{wl.name} static-scratch call {call + 1}")
+    del keep
