@@ -55,6 +55,28 @@ def _config(extra=None):
     return cfg
 
 
+def _kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("wave_attn.cu", "ptx.cuh", "exp2_poly.h"):
+        with open(os.path.join(ROOT, "block_causal_attention_wave_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _measured_traffic():
+    """DRAM bytes per attention launch from the committed ncu capture, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "round_attn_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != _kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def _measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -218,9 +240,6 @@ def run_gpu(args):
     n_keys = [sum(v for _, v in rows) for rows in table]
     flops = sum(4 * wl.tokens * nk * wl.heads * wl.head_dim for nk in n_keys)
     upd_nodes = sum(1 for n in active if n[1] > 0)
-    append_bytes = 0
-    for rows in table:
-        pass
     per_node_read = 2 * wl.tokens * wl.heads * wl.head_dim * 2
     per_node_write = 2 * math.ceil(wl.tokens / 128) * 128 * wl.heads * wl.head_dim * 2
     append_bytes = len(active) * (per_node_read + per_node_write)
@@ -322,7 +341,7 @@ def run_gpu(args):
                 "ms_per_step": round(e2e_ms, 4)},
         "roofline": {"bound": "tensor", "kernel": "round_attn_kernel<128>",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": _measured_traffic(),
                      "peak_source": f"{src} bf16_tflops (burst, cuBLAS 8192^3)",
                      "flops_per_launch": flops, "avg_launch_ms": round(attn_avg, 4)},
         "append": {"kernel": "kv_append_kernel", "avg_launch_ms": round(append_ms, 4),
@@ -375,13 +394,11 @@ def _oracle_sample(active, entries, qs, n_rows):
     oatt.round_attention(active, POLICY, wl.window, qs, entries, None,
                          {n: rows for n in active})
     dt = time.perf_counter() - t
-    n_keys = {n: (len(active) and None) for n in active}
-    flops = 0
     from oracle import cache as ocache
+    flops = 0
     for n in active:
         nk = len(ocache.key_entries(n, POLICY, wl.window, False)) * wl.tokens
         flops += 4 * len(rows) * nk * wl.heads * wl.head_dim
-    del n_keys
     return dt, flops, len(rows)
 
 
@@ -396,6 +413,7 @@ def _cores():
 
 def cpu_baseline(target_s=10.0):
     active, entries, qs = _oracle_round()
+    _oracle_sample(active, entries, qs, 4)  # first touch of the float64 inputs
     dt, _, _ = _oracle_sample(active, entries, qs, 16)
     n_rows = int(min(1024, max(16, 16 * target_s / max(dt, 1e-3))))
     dt, flops, nr = _oracle_sample(active, entries, qs, n_rows)

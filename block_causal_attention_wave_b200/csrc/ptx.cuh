@@ -174,6 +174,81 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+
+// Eight kind::f16 MMAs that together contract K = 128 (8 steps of 16), issued
+// in one block so the issuing thread spends one instruction per MMA besides
+// the descriptor arithmetic. Step k uses the low descriptor words a_lo + da[k]
+// and b_lo + db[k] (offsets in 16-byte units, compile-time constants) with the
+// shared high words a_hi / b_hi. The first step overwrites D unless
+// `accumulate` is set; the other seven accumulate.
+template <uint32_t DA, uint32_t DA_PANEL, uint32_t DB, uint32_t DB_PANEL>
+__device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                            uint32_t accumulate) {
+  // step k: +k*DA within a panel (k < 4), +DA_PANEL for the second panel
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t.reg .b32 al, bl;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\tsetp.eq.b32 t, %5, %5;\n\t"
+      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, p;\n\t"
+      "add.u32 al, %1, %7;\n\tadd.u32 bl, %3, %8;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %9;\n\tadd.u32 bl, %3, %10;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %11;\n\tadd.u32 bl, %3, %12;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %13;\n\tadd.u32 bl, %3, %14;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %15;\n\tadd.u32 bl, %3, %16;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %17;\n\tadd.u32 bl, %3, %18;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t"
+      "add.u32 al, %1, %19;\n\tadd.u32 bl, %3, %20;\n\t"
+      "mov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %6, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(accumulate), "r"(idesc),
+      "n"(1 * DA), "n"(1 * DB), "n"(2 * DA), "n"(2 * DB), "n"(3 * DA), "n"(3 * DB),
+      "n"(DA_PANEL), "n"(DB_PANEL), "n"(DA_PANEL + DA), "n"(DB_PANEL + DB),
+      "n"(DA_PANEL + 2 * DA), "n"(DB_PANEL + 2 * DB), "n"(DA_PANEL + 3 * DA),
+      "n"(DB_PANEL + 3 * DB)
+      : "memory");
+}
+
+// Eight MMAs with A from TMEM (columns a_tmem + 8k) and B from shared memory
+// (low descriptor word b_lo + k * DB), K = 128 in 8 steps of 16.
+template <uint32_t DB>
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                            uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 b;\n\t.reg .b32 bl, ta;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %5, p;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.u32 bl, %2, %6;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 16;\n\tadd.u32 bl, %2, %7;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 24;\n\tadd.u32 bl, %2, %8;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 32;\n\tadd.u32 bl, %2, %9;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 40;\n\tadd.u32 bl, %2, %10;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 48;\n\tadd.u32 bl, %2, %11;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t"
+      "add.u32 ta, %1, 56;\n\tadd.u32 bl, %2, %12;\n\tmov.b64 b, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], b, %5, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(accumulate), "r"(idesc), "n"(1 * DB), "n"(2 * DB),
+      "n"(3 * DB), "n"(4 * DB), "n"(5 * DB), "n"(6 * DB), "n"(7 * DB)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -357,24 +357,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto slot_addr = [&](uint32_t r) -> uint32_t {
           return sbase + C::kRingOff + (r % S) * C::kTileBytes;
         };
+        // Shared-memory descriptors split into a per-address low word and a
+        // constant high word (stride 1024 B between 8-row groups, sm_100
+        // version bit, 128-byte swizzle); K-steps add constants to the low word.
+        constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+        auto lo_k = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | (1u << 16); };
+        auto lo_mn = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | ((16384u >> 4) << 16); };
         // S_w = Q_w K(t)^T into TMEM columns 128 w.
         auto issue_s = [&](int w, uint32_t t) {
           const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
           const uint32_t kaddr = slot_addr(2 * t);
+          if constexpr (D == 128) {
+            mma_ss_k128<2, C::kPanelBytes / 16, 2, C::kPanelBytes / 16>(
+                tmem + C::kColS + 128 * w, lo_k(qaddr), kDescHi, lo_k(kaddr), kDescHi, C::kIdescS,
+                0u);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-            mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off),
-                   C::kIdescS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+              mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off),
+                     C::kIdescS, kk > 0 ? 1u : 0u);
+            }
           }
         };
         // O_w (+)= P_w V(t), P_w read from TMEM (bf16 in S_w's first 64 columns).
         auto issue_pv = [&](int w, uint32_t t, bool accumulate) {
           const uint32_t vaddr = slot_addr(2 * t + 1);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w + kk * 8,
-                   desc_mn(vaddr + kk * 2048), C::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w,
+                                 lo_mn(vaddr), kDescHi, C::kIdescO, accumulate ? 1u : 0u);
         };
         for (uint32_t k = 0; ok; ++k) {
           int item;
