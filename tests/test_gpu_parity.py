@@ -210,3 +210,18 @@ def test_duplicate_and_single_nodes(cuda_lib):
     ref = oracle_outputs(inp, [(1, 1)], "progressive")
     assert_close(torch_to_f64(o[:200]), ref[(1, 1)], "dup")
     del keep
+
+
+def test_wan21_same_level_round_sampled_rows(cuda_lib):
+    """Same-level policy at the Wan2.1 shapes: history read at the node's own level."""
+    rows = np.array([0, 129, 2222, 4607, 4679])
+    res = _one_round(cuda_lib, wi.WAN21, "same", 6, rows)
+    assert len(res) == 4  # (3,4)...: same-level round 6 has no refresh
+
+
+def test_long_rollout_clean_round_sampled_rows(cuda_lib):
+    """Clean policy, 40 chunks x 4680 tokens, window 6, 5 levels: a late round."""
+    rows = np.array([0, 4000, 4679])
+    rounds = osched.schedule(wi.LONG_ROLLOUT.chunks, wi.LONG_ROLLOUT.levels, "clean", 6)
+    res = _one_round(cuda_lib, wi.LONG_ROLLOUT, "clean", len(rounds) - 5, rows)
+    assert len(res) == len(rounds[len(rounds) - 5])
