@@ -42,18 +42,42 @@ import wave_inputs as wi  # noqa: E402
 
 METRIC = "wave-round attention TFLOP/s and chunk-updates/s at 1 B200; % of BF16 dense peak"
 UNIT = "TFLOP/s"
-WORKLOAD = "wan2.1-1.3b round 6 (B=7, K=4, progressive)"
-ROUND = 6
 POLICY = "progressive"
 
 
-def _config(extra=None):
-    wl = wi.WAN21
-    cfg = {"workload": WORKLOAD, "heads": wl.heads, "head_dim": wl.head_dim,
+class Spec:
+    """A timed wave round: the workload's shapes and which round of its schedule."""
+
+    def __init__(self, key, wl, round_index, label, pool_pages):
+        self.key, self.wl, self.round, self.label, self.pool_pages = (
+            key, wl, round_index, label, pool_pages)
+
+
+WORKLOADS = {
+    # Wan2.1-1.3B-shaped round (the headline): nodes (2,0) refresh, (3,1), (4,2),
+    # (5,3), (6,4); the live cache peaks near 900 pages.
+    "wan21": Spec("wan21", wi.WAN21, 6, "wan2.1-1.3b round 6 (B=7, K=4, progressive)", 2400),
+    # Wan-Streamer-shaped steady round: (33,0) refresh, (34,1), (35,2); 984-token
+    # units, 512-token prefix, 32-unit window, 24 heads.
+    "wan-streamer": Spec("wan-streamer", wi.WAN_STREAMER, 35,
+                         "wan-streamer unit round 35 (K=2, W=32, prefix 512, progressive)", 1000),
+    # Long rollout steady round: (15,0) refresh, (16,1) .. (20,5); window 6.
+    "long-rollout": Spec("long-rollout", wi.LONG_ROLLOUT, 20,
+                         "long rollout round 20 (40 chunks, K=5, W=6, progressive)", 1400),
+}
+DEFAULT_WORKLOAD = "wan21"
+# Headline constants (the CPU-baseline and reference legs time this round).
+ROUND = WORKLOADS[DEFAULT_WORKLOAD].round
+WORKLOAD = WORKLOADS[DEFAULT_WORKLOAD].label
+
+
+def _config(extra=None, spec=None):
+    spec = spec or WORKLOADS[DEFAULT_WORKLOAD]
+    wl = spec.wl
+    cfg = {"workload": spec.label, "heads": wl.heads, "head_dim": wl.head_dim,
            "tokens_per_chunk": wl.tokens, "chunks": wl.chunks, "levels": wl.levels,
-           "policy": POLICY, "round": ROUND,
-           "active_nodes": "(2,0) refresh, (3,1), (4,2), (5,3), (6,4)",
-           "l2": "inputs larger than L2 (round K/V 0.7 GB, Q 72 MB); no flush"}
+           "window": wl.window, "prefix_tokens": wl.prefix, "policy": POLICY, "round": spec.round,
+           "l2": "inputs larger than L2 (the round's K/V and Q); no flush"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -179,12 +203,13 @@ class ClockSampler:
 class Round:
     """Host-side description of the timed round, from the library's scheduler."""
 
-    def __init__(self, wave):
-        wl = wi.WAN21
-        self.wl = wl
+    def __init__(self, wave, spec=None):
+        spec = spec or WORKLOADS[DEFAULT_WORKLOAD]
+        wl = spec.wl
+        self.spec, self.wl = spec, wl
         self.rounds = wave.schedule(wl.chunks, wl.levels, POLICY, wl.window)
         self.last = wave.last_read_rounds(wl.chunks, wl.levels, POLICY, wl.window)
-        self.active = self.rounds[ROUND]
+        self.active = self.rounds[spec.round]
 
 
 def _bits_to_dev(bits, pin=False):
@@ -205,19 +230,23 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     wave.load()
-    rd = Round(wave)
+    spec = WORKLOADS[args.workload]
+    rd = Round(wave, spec)
     wl = rd.wl
     page_bytes = wave.KVCache.page_bytes(wl.heads, wl.head_dim)
-    n_pages = 2400  # 1.9 GB: the live cache peaks near 900 pages
-    pool = torch.empty(4096 + n_pages * page_bytes, dtype=torch.uint8, device="cuda")
-    kv = wave.KVCache(wl.heads, wl.head_dim, wl.tokens, wl.levels, wl.window, 0, pool=pool)
+    pool = torch.empty(4096 + spec.pool_pages * page_bytes, dtype=torch.uint8, device="cuda")
+    kv = wave.KVCache(wl.heads, wl.head_dim, wl.tokens, wl.levels, wl.window, wl.prefix,
+                      pool=pool)
     stream = torch.cuda.current_stream()
 
     def kvbits(kind, e):
-        return wi.node_tensor(kind, e[0], e[1], wl.tokens, wl.heads, wl.head_dim, wl.scale)
+        n = wl.prefix if e[0] == -1 else wl.tokens
+        return wi.node_tensor(kind, e[0], e[1], n, wl.heads, wl.head_dim, wl.scale)
 
     # Bring the cache to the start of the timed round (untimed).
-    for t in range(ROUND):
+    if wl.prefix:
+        kv.append(-1, 0, _bits_to_dev(kvbits("k", (-1, 0))), _bits_to_dev(kvbits("v", (-1, 0))))
+    for t in range(spec.round):
         for n in rd.rounds[t]:
             kv.append(n[0], n[1], _bits_to_dev(kvbits("k", n)), _bits_to_dev(kvbits("v", n)))
         for e in sorted(e for e, lr in rd.last.items() if lr == t):
@@ -367,7 +396,7 @@ def run_gpu(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": _config({"replicas": ws}),
+        "config": _config({"replicas": ws}, spec),
         "chunk_updates_per_s": round(ws * upd_nodes * K / (ms * 1e-3), 2),
         "pct_bf16_dense_peak": round(100 * value / ws / peak, 2),
         "e2e": {"value": round(ws * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
@@ -388,7 +417,7 @@ def run_gpu(args):
         "gpu_launches": K * (len(active) + 1),
         "clocks": clocks,
     }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and spec.key == DEFAULT_WORKLOAD:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -496,6 +525,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["wave", "reference"], default="wave")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
+                    help="timed round; the default is the headline Wan2.1-shaped round")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -81,8 +81,9 @@ typedef struct {
 } wave_kv_config;
 
 /* Create a paged (chunk, level) K/V cache over cfg->pool ([WF] history cache,
- * [WS] "K/V cache"). The pool holds a 4096-byte header (device status word)
- * followed by pages of 2*H*128*d bf16 values: K as [H][128][d], then V as
+ * [WS] "K/V cache"). The pool holds a 4096-byte header (the device status
+ * word at byte 0, the attention kernel's work-queue counter at byte 128) and
+ * then pages of 2*H*128*d bf16 values: K as [H][128][d], then V as
  * [H][128][d]. Page p starts at pool + data_offset + p * page_bytes. With a
  * non-NULL pool this call clears the header synchronously and needs a CUDA
  * device with sm_100. *out receives the handle; destroy it with

@@ -225,3 +225,31 @@ def test_long_rollout_clean_round_sampled_rows(cuda_lib):
     rounds = osched.schedule(wi.LONG_ROLLOUT.chunks, wi.LONG_ROLLOUT.levels, "clean", 6)
     res = _one_round(cuda_lib, wi.LONG_ROLLOUT, "clean", len(rounds) - 5, rows)
     assert len(res) == len(rounds[len(rounds) - 5])
+
+
+def test_capacity_and_alignment_errors_before_launch(cuda_lib):
+    """Rounds beyond one launch's tables, and misaligned Q, fail cleanly."""
+    import torch
+    wl = wi.Workload("cap", chunks=8000, levels=1, heads=1, head_dim=64, tokens=128)
+    kv = make_cache(cuda_lib, wl, 7300)
+    # 7200 cached level-0 history entries (reserved, not written) + the node's own:
+    # chunk 7200 at level 1 reads 7201 one-page entries > 7168 pages per launch.
+    for c in range(7200):
+        kv.alloc(c, 0)
+    kv.alloc(7200, 1)
+    q = torch.zeros(128, 1, 64, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.round_attn([(7200, 1)], "clean", q, o)
+    assert e.value.code == -7
+    nodes = [(c, 0) for c in range(65)]
+    q65 = torch.zeros(65 * 128, 1, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.round_attn(nodes, "clean", q65, torch.empty_like(q65))
+    assert e.value.code == -7
+    raw = torch.zeros(128 * 64 + 8, dtype=torch.bfloat16, device="cuda")
+    q_mis = raw[1:1 + 128 * 64].view(128, 1, 64)  # 2-byte offset
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.round_attn([(1, 0)], "clean", q_mis, o)
+    assert e.value.code == -1
+    kv.status()
