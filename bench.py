@@ -308,6 +308,10 @@ def run_gpu(args):
     barrier()
     clocks = clk.stop()
     kv.status(stream)
+    # SM clock the last timed attention launch ran at (its CTA 0's cycles / ns).
+    cyc, ns = kv.last_launch_clock(stream)
+    eff_mhz = cyc / ns * 1e3 if ns > 0 else None
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
     ms_local = t0.elapsed_time(t1)
     attn_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
     ms = reduce_max(ms_local, "cuda" if ws > 1 else None)
@@ -408,7 +412,12 @@ def run_gpu(args):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": _measured_traffic(),
                      "peak_source": f"{src} bf16_tflops (burst, cuBLAS 8192^3)",
-                     "flops_per_launch": flops, "avg_launch_ms": round(attn_avg, 4)},
+                     "flops_per_launch": flops, "avg_launch_ms": round(attn_avg, 4),
+                     "effective_sm_mhz": round(eff_mhz, 1) if eff_mhz else None,
+                     "per_clock_frac": (round(achieved / (sms * 8192 * eff_mhz * 1e-6), 4)
+                                        if eff_mhz else None),
+                     "per_clock_note": "achieved / (SMs x 8192 dense bf16 FLOP/clk x the "
+                                       "effective SM clock of the last timed launch)"},
         "append": {"kernel": "kv_append_kernel", "avg_launch_ms": round(append_ms, 4),
                    "achieved_gbs": round(append_bytes / len(active) / (append_ms * 1e-3) / 1e9, 1),
                    "peak_gbs": peaks["hbm_gbs"],

@@ -67,6 +67,9 @@ _SIGS = {
                                                       ctypes.c_void_p, ctypes.c_void_p,
                                                       ctypes.c_void_p]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_kv_last_launch_clock": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.POINTER(ctypes.c_int64),
+                                                 ctypes.POINTER(ctypes.c_int64)]),
     "wave_schedule": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.POINTER(Node), ctypes.c_int32,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
@@ -258,3 +261,11 @@ class KVCache:
     def status(self, stream=None):
         """Synchronise and raise WaveError if a kernel timed out."""
         _check(self.lib.wave_kv_status(self.h, _stream_handle(stream)))
+
+    def last_launch_clock(self, stream=None):
+        """(SM cycles, nanoseconds) of the last attention launch's first CTA;
+        cycles / ns is the SM clock in GHz that the launch ran at."""
+        cyc, ns = ctypes.c_int64(0), ctypes.c_int64(0)
+        _check(self.lib.wave_kv_last_launch_clock(self.h, _stream_handle(stream),
+                                                  ctypes.byref(cyc), ctypes.byref(ns)))
+        return cyc.value, ns.value

@@ -80,6 +80,7 @@ struct AttnParams {
   uint16_t* out;      // O, bf16 [rows][H][d]
   int32_t* status;    // device status word (pool header)
   int32_t* counter;   // work-queue counter, zero at launch (pool header)
+  int64_t* clock_out; // CTA 0's SM cycles and nanoseconds (pool header)
   float scale_log2;   // log2(e) / sqrt(d)
   int32_t heads;
   int32_t n_nodes;
@@ -143,7 +144,7 @@ struct Bars {
   static constexpr int kS = Cfg<D>::kSlots;
   static constexpr int RING_FULL = B_RING_FULL, RING_EMPTY = RING_FULL + kS,
                        COUNT = RING_EMPTY + kS;
-  static_assert(COUNT * 8 + 16 + 4 * kItemSlots <= 512, "barrier area");
+  static_assert(COUNT * 8 + 16 + 4 * kItemSlots <= 448, "barrier area");  // 448..463: clock
 };
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
@@ -242,6 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA 0 times itself in SM cycles and in nanoseconds (start kept in shared
+  // memory): their ratio is the SM clock the launch actually ran at.
+  volatile int64_t* clock_start = reinterpret_cast<volatile int64_t*>(smem + C::kBarOff + 448);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    clock_start[0] = clock64();
+    clock_start[1] = (int64_t)globaltimer_ns();
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q_FULL), 1);
@@ -592,6 +600,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kCols);
   }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.clock_out[0] = clock64() - clock_start[0];
+    p.clock_out[1] = (int64_t)globaltimer_ns() - clock_start[1];
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -682,6 +694,7 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
   prm.out = static_cast<uint16_t*>(O);
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
   prm.counter = counter;
+  prm.clock_out = reinterpret_cast<int64_t*>(static_cast<char*>(kv->cfg.pool) + 256);
   prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   prm.heads = H;
   prm.q_rows = T;

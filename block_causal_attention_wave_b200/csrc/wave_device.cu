@@ -151,6 +151,25 @@ int launch_append(wave_kv* kv, const wave_entry& ent, const void* K, const void*
 
 }  // namespace wavei
 
+extern "C" int wave_kv_last_launch_clock(wave_kv* kv, void* stream, int64_t* cycles,
+                                         int64_t* ns) {
+  using namespace wavei;
+  clear_error();
+  if (!kv || !cycles || !ns) return fail(WAVE_ERR_ARG, "NULL argument");
+  *cycles = 0;
+  *ns = 0;
+  if (!kv->on_device) return WAVE_OK;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int64_t words[2] = {0, 0};
+  e = cudaMemcpy(words, static_cast<char*>(kv->cfg.pool) + 256, sizeof words,
+                 cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clock words)");
+  *cycles = words[0];
+  *ns = words[1];
+  return WAVE_OK;
+}
+
 extern "C" int wave_kv_status(wave_kv* kv, void* stream) {
   using namespace wavei;
   clear_error();

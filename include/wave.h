@@ -82,7 +82,8 @@ typedef struct {
 
 /* Create a paged (chunk, level) K/V cache over cfg->pool ([WF] history cache,
  * [WS] "K/V cache"). The pool holds a 4096-byte header (the device status
- * word at byte 0, the attention kernel's work-queue counter at byte 128) and
+ * word at byte 0, the attention kernel's work-queue counter at byte 128, the
+ * last attention launch's clock words at bytes 256..271) and
  * then pages of 2*H*128*d bf16 values: K as [H][128][d], then V as
  * [H][128][d]. Page p starts at pool + data_offset + p * page_bytes. With a
  * non-NULL pool this call clears the header synchronously and needs a CUDA
@@ -171,6 +172,15 @@ int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active, int3
  * without ordering) race on it and give undefined results. */
 int wave_round_attn_static_scratch(wave_kv* kv, const wave_node* active, int32_t n_active,
                                    int32_t policy, const void* Q, void* O, void* stream);
+
+/* Synchronise `stream`, then read the clock words of the last attention
+ * launch on this pool: *cycles = SM clock cycles and *ns = nanoseconds
+ * (%globaltimer) between the start and the end of the launch's first CTA, as
+ * int64 at bytes 256 and 264 of the pool header. *cycles / *ns (GHz) is the
+ * SM clock the tensor-core kernel actually ran at; clock readings sampled by
+ * the driver every few milliseconds miss short clock reductions. Both are 0
+ * before the first launch and for a host-only handle. Errors: ARG, CUDA. */
+int wave_kv_last_launch_clock(wave_kv* kv, void* stream, int64_t* cycles, int64_t* ns);
 
 /* Synchronise `stream`, then read and clear the pool's device status word.
  * Returns WAVE_OK, WAVE_ERR_TIMEOUT if a kernel gave up on a bounded wait

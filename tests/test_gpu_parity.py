@@ -253,3 +253,21 @@ def test_capacity_and_alignment_errors_before_launch(cuda_lib):
         kv.round_attn([(1, 0)], "clean", q_mis, o)
     assert e.value.code == -1
     kv.status()
+
+
+def test_launch_clock_words(cuda_lib):
+    """The attention launch records its first CTA's SM cycles and nanoseconds;
+    before any launch both words are zero."""
+    import torch
+    wl = dataclasses.replace(wi.TINY, tokens=200, head_dim=128)
+    inp = Inputs(wl)
+    kv = make_cache(cuda_lib, wl, 16)
+    assert kv.last_launch_clock() == (0, 0)
+    keep = [append(kv, inp, e) for e in ((0, 0), (1, 1))]
+    q = queries(inp, [(1, 1)])
+    kv.round_attn([(1, 1)], "progressive", q, torch.empty_like(q))
+    kv.status()
+    cyc, ns = kv.last_launch_clock()
+    assert cyc > 0 and ns > 0
+    assert 0.2 < cyc / ns < 2.5, (cyc, ns)  # GHz
+    del keep
