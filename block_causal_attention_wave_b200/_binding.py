@@ -67,6 +67,10 @@ _SIGS = {
                                                       ctypes.c_void_p, ctypes.c_void_p,
                                                       ctypes.c_void_p]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_kv_append_batch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Node),
+                                            ctypes.POINTER(ctypes.c_void_p),
+                                            ctypes.POINTER(ctypes.c_void_p),
+                                            ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
     "wave_kv_last_launch_clock": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.POINTER(ctypes.c_int64),
                                                  ctypes.POINTER(ctypes.c_int64)]),
@@ -217,6 +221,19 @@ class KVCache:
         n = K.shape[0]
         _check(self.lib.wave_kv_append(self.h, chunk, level, ctypes.c_void_p(K.data_ptr()),
                                        ctypes.c_void_p(V.data_ptr()), n, _stream_handle(stream)))
+
+    def append_batch(self, entries, Ks, Vs, stream=None):
+        """Append several entries with one kernel launch; pages are taken in
+        list order, as the same appends one by one would take them."""
+        n = len(entries)
+        if not (len(Ks) == len(Vs) == n):
+            raise ValueError("one K and one V per entry")
+        ptr = ctypes.c_void_p * max(n, 1)
+        ks = ptr(*[K.data_ptr() for K in Ks])
+        vs = ptr(*[V.data_ptr() for V in Vs])
+        nt = (ctypes.c_int32 * max(n, 1))(*[K.shape[0] for K in Ks])
+        _check(self.lib.wave_kv_append_batch(self.h, n, _nodes(entries), ks, vs, nt,
+                                             _stream_handle(stream)))
 
     def release(self, chunk, level):
         _check(self.lib.wave_kv_release(self.h, chunk, level))

@@ -18,58 +18,73 @@ namespace wavei {
 
 namespace {
 
-constexpr int kMaxEntryPages = 4096;  // 512K tokens per entry
-
-struct AppendParams {
-  const uint4* k;
+// One launch copies every entry of an append call. The work unit is a tile:
+// one page's 128 token rows of one head, of K or of V (16 KB at d = 64, 32 KB
+// at d = 128), which is one contiguous run of the destination page. A block
+// takes one tile: the tile's coordinates cost one search over at most 64
+// entries and two small divisions per block, nothing per element.
+struct AppendEntry {
+  const uint4* k;    // [ntokens][H][d] bf16 as 16-byte vectors
   const uint4* v;
-  uint8_t* data;        // pool + data_offset
-  int64_t page_bytes;
   int32_t ntokens;
-  int32_t heads;
   int32_t n_pages;
-  int32_t vec_per_row;  // head_dim / 8 (16-byte vectors per token row)
-  int32_t pages[kMaxEntryPages];
+  int32_t page0;     // index of the entry's first page in `pages`
+  int32_t tile0;     // index of the entry's first tile
 };
 
-// One 16-byte vector per thread step. The linear index walks the DESTINATION in
-// order (K then V; page; head; token-in-page; vector), so stores are fully
-// contiguous; each group of vec_per_row threads reads one 128/256-byte token
-// row of the source, which keeps loads sector-efficient as well.
-__global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
-  const int64_t per_head = (int64_t)WAVE_PAGE_TOKENS * p.vec_per_row;
-  const int64_t per_page = per_head * p.heads;
-  const int64_t per_kv = per_page * p.n_pages;
-  const int64_t total = 2 * per_kv;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  constexpr int kUnroll = 4;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x * kUnroll + threadIdx.x; base < total;
-       base += stride * kUnroll) {
-    uint4 val[kUnroll];
-    uint4* dst[kUnroll];
+struct AppendParams {
+  uint8_t* data;        // pool + data_offset
+  int64_t page_bytes;
+  int32_t heads;
+  int32_t vec_per_row;  // head_dim / 8 (16-byte vectors per token row): 8 or 16
+  int32_t log2_vec;
+  int32_t n_entries;
+  int32_t n_tiles;
+  int32_t pad;
+  AppendEntry e[WAVE_MAX_APPEND_ENTRIES];
+  int32_t pages[WAVE_MAX_APPEND_PAGES];
+};
+static_assert(sizeof(AppendParams) <= 32760, "kernel parameter space is 32 KB");
+
+constexpr int kAppendThreads = 256;
+constexpr int kAppendPer = WAVE_PAGE_TOKENS * 16 / kAppendThreads;  // vectors per thread, d = 128
+
+// Thread t moves vectors t, t + 256, ... of the tile: every group of
+// vec_per_row threads reads one 128/256-byte token row of the source (its
+// head's slice), and the block's stores fill the tile's bytes in order. Loads
+// are all issued before the stores. Rows past the entry's last token are
+// written as zeros.
+__global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(
+    const __grid_constant__ AppendParams p) {
+  const int tile = blockIdx.x;
+  if (tile >= p.n_tiles) return;
+  int ei = 0;
+  while (ei + 1 < p.n_entries && tile >= p.e[ei + 1].tile0) ++ei;
+  const AppendEntry& en = p.e[ei];
+  int local = tile - en.tile0;
+  const int per_kv = en.n_pages * p.heads;
+  const int kv = local >= per_kv;
+  local -= kv * per_kv;
+  const int pi = local / p.heads;
+  const int h = local - pi * p.heads;
+  const int per_tile = WAVE_PAGE_TOKENS * p.vec_per_row;
+  const uint4* src = kv ? en.v : en.k;
+  uint4* dst = reinterpret_cast<uint4*>(p.data + (int64_t)p.pages[en.page0 + pi] * p.page_bytes) +
+               ((int64_t)kv * p.heads + h) * per_tile;
+  const int token0 = pi * WAVE_PAGE_TOKENS;
+  uint4 val[kAppendPer];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t i = base + (int64_t)u * blockDim.x;
-      dst[u] = nullptr;
-      if (i >= total) continue;
-      int kv = i >= per_kv;
-      int64_t j = i - kv * per_kv;
-      int pi = (int)(j / per_page);
-      int64_t r = j - (int64_t)pi * per_page;
-      int h = (int)(r / per_head);
-      int64_t r2 = r - (int64_t)h * per_head;
-      int t = (int)(r2 / p.vec_per_row);
-      int c = (int)(r2 - (int64_t)t * p.vec_per_row);
-      int token = pi * WAVE_PAGE_TOKENS + t;
-      const uint4* src = kv ? p.v : p.k;
-      val[u] = make_uint4(0, 0, 0, 0);
-      if (token < p.ntokens) val[u] = __ldg(src + ((int64_t)token * p.heads + h) * p.vec_per_row + c);
-      uint8_t* page = p.data + (int64_t)p.pages[pi] * p.page_bytes;
-      dst[u] = reinterpret_cast<uint4*>(page) + ((int64_t)kv * p.heads + h) * per_head + r2;
-    }
+  for (int u = 0; u < kAppendPer; ++u) {
+    const int i = threadIdx.x + u * kAppendThreads;
+    val[u] = make_uint4(0, 0, 0, 0);
+    const int token = token0 + (i >> p.log2_vec);
+    if (i < per_tile && token < en.ntokens)
+      val[u] = __ldg(src + ((int64_t)token * p.heads + h) * p.vec_per_row + (i & (p.vec_per_row - 1)));
+  }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (dst[u]) *dst[u] = val[u];
+  for (int u = 0; u < kAppendPer; ++u) {
+    const int i = threadIdx.x + u * kAppendThreads;
+    if (i < per_tile) dst[i] = val[u];
   }
 }
 
@@ -124,26 +139,31 @@ int device_init(wave_kv* kv) {
   return WAVE_OK;
 }
 
-int launch_append(wave_kv* kv, const wave_entry& ent, const void* K, const void* V,
-                  int32_t ntokens, void* stream) {
-  if ((int)ent.pages.size() > kMaxEntryPages)
-    return fail(WAVE_ERR_CAPACITY, "entry of %d pages exceeds %d", (int)ent.pages.size(),
-                kMaxEntryPages);
+int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,
+                  const void* const* K, const void* const* V, void* stream) {
   static thread_local AppendParams p;  // large: keep off the stack; launch copies it
-  p.k = static_cast<const uint4*>(K);
-  p.v = static_cast<const uint4*>(V);
+  if (n < 1 || n > WAVE_MAX_APPEND_ENTRIES) return fail(WAVE_ERR_ARG, "bad entry count %d", n);
   p.data = static_cast<uint8_t*>(kv->cfg.pool) + kv->data_offset;
   p.page_bytes = kv->page_bytes;
-  p.ntokens = ntokens;
   p.heads = kv->cfg.heads;
-  p.n_pages = (int32_t)ent.pages.size();
   p.vec_per_row = kv->cfg.head_dim / 8;
-  std::memcpy(p.pages, ent.pages.data(), ent.pages.size() * sizeof(int32_t));
-  int64_t total = 2LL * p.n_pages * WAVE_PAGE_TOKENS * p.heads * p.vec_per_row;
-  int64_t blocks = (total + 256 * 4 - 1) / (256 * 4);
-  int64_t cap = (int64_t)kv->num_sms * 8;
-  if (blocks > cap) blocks = cap;
-  kv_append_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  p.log2_vec = p.vec_per_row == 16 ? 4 : 3;
+  p.n_entries = n;
+  int32_t pages = 0, tiles = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const wave_entry& ent = *entries[i];
+    const int32_t np = (int32_t)ent.pages.size();
+    if (pages + np > WAVE_MAX_APPEND_PAGES)
+      return fail(WAVE_ERR_CAPACITY, "more than %d pages in one append", WAVE_MAX_APPEND_PAGES);
+    p.e[i] = AppendEntry{static_cast<const uint4*>(K[i]), static_cast<const uint4*>(V[i]),
+                         ent.ntokens, np, pages, tiles};
+    std::memcpy(p.pages + pages, ent.pages.data(), np * sizeof(int32_t));
+    pages += np;
+    tiles += 2 * np * p.heads;
+  }
+  p.n_tiles = tiles;
+  if (tiles == 0) return WAVE_OK;
+  kv_append_kernel<<<(unsigned)tiles, kAppendThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kv_append_kernel launch");
   return WAVE_OK;

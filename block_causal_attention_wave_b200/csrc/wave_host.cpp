@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <set>
 #include <string>
 
 #include "wave_internal.h"
@@ -165,9 +166,9 @@ int wave_kv_pool_layout(const wave_kv* kv, int64_t* page_bytes, int64_t* data_of
   return WAVE_OK;
 }
 
-int wave_kv_alloc(wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens) {
-  clear_error();
-  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+namespace wavei {
+// Shape and existence checks of wave_kv_alloc, without taking pages.
+static int check_new_entry(const wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens) {
   if (chunk == WAVE_PREFIX_CHUNK) {
     if (level != 0 || ntokens != kv->cfg.prefix_tokens || ntokens < 1)
       return fail(WAVE_ERR_ARG, "prefix must be level 0 with prefix_tokens (%d) tokens",
@@ -179,8 +180,17 @@ int wave_kv_alloc(wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens) {
       return fail(WAVE_ERR_ARG, "entry needs tokens_per_chunk (%d) tokens, got %d",
                   kv->cfg.tokens_per_chunk, ntokens);
   }
+  if (kv->entries.count(std::make_pair(chunk, level)))
+    return fail(WAVE_ERR_EXISTS, "(%d, %d) already cached", chunk, level);
+  return WAVE_OK;
+}
+}  // namespace wavei
+
+int wave_kv_alloc(wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens) {
+  clear_error();
+  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+  if (int rc = check_new_entry(kv, chunk, level, ntokens)) return rc;
   auto key = std::make_pair(chunk, level);
-  if (kv->entries.count(key)) return fail(WAVE_ERR_EXISTS, "(%d, %d) already cached", chunk, level);
   int32_t need = (ntokens + kPageTokens - 1) / kPageTokens;
   if ((int64_t)need > (int64_t)kv->free_pages.size())
     return fail(WAVE_ERR_NO_PAGES, "need %d pages, %zu free", need, kv->free_pages.size());
@@ -216,18 +226,57 @@ int wave_kv_free_pages(const wave_kv* kv, int32_t* n) {
 
 int wave_kv_append(wave_kv* kv, int32_t chunk, int32_t level, const void* K, const void* V,
                    int32_t ntokens, void* stream) {
+  const wave_node e{chunk, level};
+  return wave_kv_append_batch(kv, 1, &e, &K, &V, &ntokens, stream);
+}
+
+int wave_kv_append_batch(wave_kv* kv, int32_t n_entries, const wave_node* entries,
+                         const void* const* K, const void* const* V, const int32_t* ntokens,
+                         void* stream) {
   clear_error();
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL) cannot append");
-  if (!K || !V || ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V)) & 15))
-    return fail(WAVE_ERR_ARG, "K and V must be non-NULL and 16-byte aligned");
-  int rc = wave_kv_alloc(kv, chunk, level, ntokens);
-  if (rc) return rc;
-  const wave_entry& e = kv->entries.at(std::make_pair(chunk, level));
-  rc = launch_append(kv, e, K, V, ntokens, stream);
+  if (n_entries < 0 || (n_entries > 0 && (!entries || !K || !V || !ntokens)))
+    return fail(WAVE_ERR_ARG, "bad arguments");
+  if (n_entries > WAVE_MAX_APPEND_ENTRIES)
+    return fail(WAVE_ERR_CAPACITY, "%d entries exceed %d per append call", n_entries,
+                WAVE_MAX_APPEND_ENTRIES);
+  // Check everything before taking any page.
+  int64_t need = 0;
+  std::set<std::pair<int32_t, int32_t>> seen;
+  for (int32_t i = 0; i < n_entries; ++i) {
+    if (!K[i] || !V[i] || ((reinterpret_cast<uintptr_t>(K[i]) | reinterpret_cast<uintptr_t>(V[i])) & 15))
+      return fail(WAVE_ERR_ARG, "K and V of entry %d must be non-NULL and 16-byte aligned", i);
+    if (int rc = check_new_entry(kv, entries[i].chunk, entries[i].level, ntokens[i])) return rc;
+    if (!seen.insert(std::make_pair(entries[i].chunk, entries[i].level)).second)
+      return fail(WAVE_ERR_ARG, "(%d, %d) named twice in one append call", entries[i].chunk,
+                  entries[i].level);
+    need += (ntokens[i] + kPageTokens - 1) / kPageTokens;
+  }
+  if (need > WAVE_MAX_APPEND_PAGES)
+    return fail(WAVE_ERR_CAPACITY, "%lld pages exceed %d per append call", (long long)need,
+                WAVE_MAX_APPEND_PAGES);
+  if (need > (int64_t)kv->free_pages.size())
+    return fail(WAVE_ERR_NO_PAGES, "need %lld pages, %zu free", (long long)need,
+                kv->free_pages.size());
+  std::vector<const wave_entry*> ents;
+  ents.reserve(n_entries);
+  for (int32_t i = 0; i < n_entries; ++i) {
+    int rc = wave_kv_alloc(kv, entries[i].chunk, entries[i].level, ntokens[i]);
+    if (rc) {  // cannot happen after the checks above; undo all the same
+      std::string keep = g_detail;
+      for (int32_t j = 0; j < i; ++j) wave_kv_release(kv, entries[j].chunk, entries[j].level);
+      g_detail = keep;
+      return rc;
+    }
+    ents.push_back(&kv->entries.at(std::make_pair(entries[i].chunk, entries[i].level)));
+  }
+  if (n_entries == 0) return WAVE_OK;
+  int rc = launch_append(kv, n_entries, ents.data(), K, V, stream);
   if (rc) {
     std::string keep = g_detail;
-    wave_kv_release(kv, chunk, level);
+    for (int32_t i = 0; i < n_entries; ++i)
+      wave_kv_release(kv, entries[i].chunk, entries[i].level);
     g_detail = keep;
   }
   return rc;

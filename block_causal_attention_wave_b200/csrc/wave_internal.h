@@ -57,7 +57,9 @@ int check_query_node(const wave_kv* kv, wave_node node);
 
 // Device halves (defined in .cu files).
 int device_init(wave_kv* kv);
-int launch_append(wave_kv* kv, const wave_entry& e, const void* K, const void* V,
-                  int32_t ntokens, void* stream);
+// One kernel launch copying the K/V of n entries (already allocated) into
+// their pages.
+int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,
+                  const void* const* K, const void* const* V, void* stream);
 
 }  // namespace wavei

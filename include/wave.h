@@ -57,6 +57,8 @@ extern "C" {
 #define WAVE_PREFIX_CHUNK  (-1)  /* chunk id of the always-visible prefix     */
 #define WAVE_MAX_NODES     64    /* active nodes per wave_round_attn call     */
 #define WAVE_MAX_PAGES_PER_ROUND 7168 /* key pages summed over a call's nodes */
+#define WAVE_MAX_APPEND_ENTRIES 64  /* entries per wave_kv_append_batch call  */
+#define WAVE_MAX_APPEND_PAGES 7168   /* pages summed over one append call       */
 
 typedef struct wave_kv wave_kv; /* opaque; owned by the library */
 
@@ -111,10 +113,26 @@ int wave_kv_alloc(wave_kv* kv, int32_t chunk, int32_t level, int32_t ntokens);
  * 16-byte aligned, caller-owned) into the new pages with one kernel on stream;
  * the unused tail of the last page is zero-filled. This is the in-round K/V
  * delivery of [WF] and the local-cache write of [WS] "pre-sharded".
- * Errors: as wave_kv_alloc, plus ARG for misaligned K/V and CUDA; on any error
- * no pages stay taken. */
+ * Errors: as wave_kv_alloc, plus ARG for misaligned K/V, CAPACITY for more
+ * than WAVE_MAX_APPEND_PAGES pages, and CUDA; on any error no pages stay
+ * taken. */
 int wave_kv_append(wave_kv* kv, int32_t chunk, int32_t level, const void* K, const void* V,
                    int32_t ntokens, void* stream);
+
+/* wave_kv_append for n_entries entries in ONE kernel launch (the round's
+ * appends of [WF] in-round delivery, batched). Entry i is (entries[i].chunk,
+ * entries[i].level) with K[i], V[i] (device, bf16 [ntokens[i]][H][d],
+ * contiguous, 16-byte aligned, caller-owned); `entries`, `K`, `V` and
+ * `ntokens` are host arrays of n_entries elements. Every entry is checked
+ * first; then pages are taken in list order, exactly as n_entries
+ * wave_kv_append calls in that order would take them, and the pages receive
+ * the same bytes. Limits: n_entries <= WAVE_MAX_APPEND_ENTRIES and total pages
+ * <= WAVE_MAX_APPEND_PAGES (else CAPACITY). Errors: ARG (including an entry
+ * named twice), EXISTS, NO_PAGES, CAPACITY, CUDA; on any error no pages stay
+ * taken. */
+int wave_kv_append_batch(wave_kv* kv, int32_t n_entries, const wave_node* entries,
+                         const void* const* K, const void* const* V, const int32_t* ntokens,
+                         void* stream);
 
 /* Return the pages of (chunk, level) to the free set. Host only; the caller
  * must not release an entry that queued device work still reads (all library

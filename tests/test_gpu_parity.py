@@ -22,8 +22,10 @@ from wave_testlib import (Inputs, append, assert_close, bits_to_torch, make_cach
 pytestmark = pytest.mark.gpu
 
 
-def _rollout_and_check(wave, wl, pol, check_rounds=None, rows_per_node=None, pages=4000):
-    """Drive a full rollout through the library; check outputs and tables."""
+def _rollout_and_check(wave, wl, pol, check_rounds=None, rows_per_node=None, pages=4000,
+                       batch=False):
+    """Drive a full rollout through the library; check outputs and tables.
+    With batch=True each round's entries go through one batched append."""
     import torch
     inp = Inputs(wl)
     kv = make_cache(wave, wl, pages)
@@ -36,7 +38,12 @@ def _rollout_and_check(wave, wl, pol, check_rounds=None, rows_per_node=None, pag
     keep = []
     results = []
     for t, active in enumerate(rounds):
-        for n in active:
+        if batch:
+            ks = [bits_to_torch(inp.bits("k", *n)) for n in active]
+            vs = [bits_to_torch(inp.bits("v", *n)) for n in active]
+            kv.append_batch(active, ks, vs)
+            keep.append((ks, vs))
+        for n in ([] if batch else active):
             keep.append(append(kv, inp, n))
         assert kv.gather_table(active, pol) == want_tables[t][1], f"round {t} table"
         if check_rounds is None or t in check_rounds:
@@ -271,3 +278,73 @@ def test_launch_clock_words(cuda_lib):
     assert cyc > 0 and ns > 0
     assert 0.2 < cyc / ns < 2.5, (cyc, ns)  # GHz
     del keep
+
+
+@pytest.mark.parametrize("pol", wi.POLICIES)
+def test_tiny_all_rounds_batched_append(cuda_lib, pol):
+    """The same rollout with each round's appends in one batched launch."""
+    _rollout_and_check(cuda_lib, dataclasses.replace(wi.TINY, tokens=300, prefix=200), pol,
+                       batch=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_append_batch_bytes_exact(cuda_lib, d):
+    """A batched append (prefix + ragged entries) takes the pages that the same
+    appends one by one take and writes the same bytes: each page [H][128][d]
+    of K then V, rows past the entry's tokens zero."""
+    import torch
+    wl = wi.Workload("batch", chunks=3, levels=2, heads=3, head_dim=d, tokens=300, prefix=130)
+    inp = Inputs(wl)
+    entries = [(-1, 0), (0, 2), (1, 1), (0, 0)]
+    kb = make_cache(cuda_lib, wl, 32)
+    ks = [bits_to_torch(inp.bits("k", *e)) for e in entries]
+    vs = [bits_to_torch(inp.bits("v", *e)) for e in entries]
+    kb.alloc(2, 1)  # pages 0..2 taken first
+    kb.append_batch(entries, ks, vs)
+    ks1 = make_cache(cuda_lib, wl, 32)
+    ks1.alloc(2, 1)
+    keep = [append(ks1, inp, e) for e in entries]
+    torch.cuda.synchronize()
+    page_bytes, off, _ = kb.layout()
+    pool, pool1 = kb.pool.cpu().numpy(), ks1.pool.cpu().numpy()
+    n_pre, n_own = (wl.prefix + 127) // 128, (wl.tokens + 127) // 128
+    for e in entries[1:]:
+        (rows,) = kb.gather_table([e], "clean")
+        assert [rows] == ks1.gather_table([e], "clean")
+        spans = [((-1, 0), rows[:n_pre], wl.prefix), (e, rows[-n_own:], wl.tokens)]
+        for ent, own, ntok in spans:
+            for kind, kvi in (("k", 0), ("v", 1)):
+                src = inp.bits(kind, *ent)
+                for pi, (page, valid) in enumerate(own):
+                    base = off + page * page_bytes + kvi * wl.heads * 128 * d * 2
+                    blk = pool[base:base + wl.heads * 128 * d * 2].view(np.uint16)
+                    blk1 = pool1[base:base + wl.heads * 128 * d * 2].view(np.uint16)
+                    np.testing.assert_array_equal(blk, blk1)
+                    blk = blk.reshape(wl.heads, 128, d)
+                    want = np.zeros_like(blk)
+                    n = min(128, ntok - pi * 128)
+                    want[:, :n, :] = src[pi * 128:pi * 128 + n].transpose(1, 0, 2)
+                    np.testing.assert_array_equal(blk, want)
+                    assert valid == n
+    del keep
+
+
+def test_append_batch_errors_take_nothing(cuda_lib):
+    import torch
+    wl = wi.Workload("batch-err", chunks=4, levels=1, heads=1, head_dim=64, tokens=128)
+    kv = make_cache(cuda_lib, wl, 3)
+    k = torch.zeros(128, 1, 64, dtype=torch.bfloat16, device="cuda")
+    free0 = kv.free_pages()
+    cases = [([(0, 1), (0, 1)], -1),                  # named twice
+             ([(0, 1), (1, 1), (2, 1), (3, 1)], -3),  # 4 pages, 3 free
+             ([(c, 0) for c in range(65)], -7)]       # more entries than one call takes
+    for entries, code in cases:
+        with pytest.raises(cuda_lib.WaveError) as e:
+            kv.append_batch(entries, [k] * len(entries), [k] * len(entries))
+        assert e.value.code == code, entries
+        assert kv.free_pages() == free0
+    kv.append_batch([(0, 1)], [k], [k])
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.append_batch([(1, 1), (0, 1)], [k, k], [k, k])
+    assert e.value.code == -6 and kv.free_pages() == free0 - 1
+    kv.status()

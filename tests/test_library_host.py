@@ -116,6 +116,12 @@ def test_error_paths(lib):
     with pytest.raises(wave.WaveError) as e:
         kv.alloc(-1, 0, 10)  # no prefix configured
     assert e.value.code == -1
+    import torch
+    k = torch.zeros(200, 2, 64, dtype=torch.bfloat16)
+    free = kv.free_pages()
+    with pytest.raises(wave.WaveError) as e:  # a host-only handle has no device to copy to
+        kv.append_batch([(3, 1)], [k], [k], stream=0)
+    assert e.value.code == -1 and kv.free_pages() == free
     with pytest.raises(wave.WaveError) as e:
         wave.KVCache(2, 96, 32, 2, pool=None, pool_bytes=1 << 20)
     assert e.value.code == -8
