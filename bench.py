@@ -147,14 +147,20 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, path: str | None = None):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.f = None
+        self.temporary = path is None
+        if path is None:
+            import tempfile
+            fd, path = tempfile.mkstemp(prefix=f"wave_clocks_rank{device_index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
@@ -165,16 +171,21 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.15)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        return self.summary()
+        out = None
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+            out = self.summary()
+        elif getattr(self, "f", None) is not None:
+            self.f.close()
+        if self.temporary and os.path.exists(self.path):
+            os.remove(self.path)
+        return out
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -298,7 +309,7 @@ def run_gpu(args):
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = ClockSampler(local)
+    clk = ClockSampler(local, args.clocks_csv.format(rank=rank) if args.clocks_csv else None)
     clk.start()
     barrier()
     torch.cuda.synchronize()
@@ -530,6 +541,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["wave", "reference"], default="wave")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the raw nvidia-smi samples here ({rank} is replaced); "
+                         "default: a temporary file")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
                     help="timed round; the default is the headline Wan2.1-shaped round")
     args = ap.parse_args(argv)
