@@ -18,6 +18,8 @@ What it computes, each part written as the plain definition from the pages:
                                list, in float64 (Wave Forcing page, "Key
                                Findings": chunk-wise causal attention over
                                earlier, cleaner chunks).
+* ``projection``            -- a node's Q, K, V = X W^T split by (Q/K/V, head),
+                               in float64 (the K/V of in-round delivery).
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
 against something other than itself (brute-force dense masks, closed forms,
@@ -25,4 +27,4 @@ torch's CPU attention, exhaustive search). Absolute attention values printed by
 the pages: none exist, so that part is "parity unpinned" against the pages and
 pinned only by the mathematics.
 """
-from . import policy, schedule, cache, attention  # noqa: F401
+from . import policy, schedule, cache, attention, projection  # noqa: F401
