@@ -86,7 +86,7 @@ def _config(extra=None, spec=None):
 def _kernel_source_hash():
     import hashlib
     h = hashlib.sha256()
-    for name in ("wave_attn.cu", "ptx.cuh", "exp2_poly.h"):
+    for name in ("wave_attn.cu", "ptx.cuh", "exp2_poly.h", "wave_sync.cuh"):
         with open(os.path.join(ROOT, "block_causal_attention_wave_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -338,6 +338,43 @@ def run_gpu(args):
     # median drops the first step, which starts from an idle GPU.
     append_ms = statistics.median(c.elapsed_time(a) for c, a in zip(ev_c, ev_a))
 
+    # ---- fused QKV projection + K/V append of the round's nodes (the step
+    # that produces the K/V the round appends), random Wan2.1-shaped weights:
+    # X [T][C] per node, W [3 H d][C]. A sleep kernel keeps the GPU busy while
+    # the host enqueues, so the events see only the launches.
+    proj = None
+    if wl.head_dim in (64, 128) and spec.key == DEFAULT_WORKLOAD:
+        dim = 1536  # Wan2.1-1.3B hidden size
+        xs = [_bits_to_dev(wi.hidden_states(n[0], n[1], wl.tokens, dim)) for n in active]
+        wqkv = _bits_to_dev(wi.qkv_weight(wl.heads, wl.head_dim, dim))
+        qp = torch.empty(wl.tokens, wl.heads, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+
+        def proj_round():
+            for n, x in zip(active, xs):
+                kv.qkv_append(n[0], n[1], x, wqkv, qp, stream)
+            for n in active:
+                kv.release(*n)
+
+        proj_round()
+        torch.cuda.synchronize()
+        reps = 5
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(3e6))
+        pa.record(stream)
+        for _ in range(reps):
+            proj_round()
+        pb.record(stream)
+        torch.cuda.synchronize()
+        kv.status(stream)
+        p_ms = pa.elapsed_time(pb) / (reps * len(active))
+        p_flops = 2 * wl.tokens * 3 * wl.heads * wl.head_dim * dim
+        proj = {"kernel": "qkv_append_kernel", "what": "Q,K,V = X W^T per node, K/V written "
+                "into the node's new pages in the epilogue", "dim": dim,
+                "flops_per_launch": p_flops, "avg_launch_ms": round(p_ms, 4),
+                "achieved": round(p_flops / (p_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "frac": round(p_flops / (p_ms * 1e-3) / 1e12 / _measured_peaks()[0]["bf16_tflops"],
+                              4)}
+
     # ---- end to end through the public API with host buffers. Every step copies
     # its Q and the round's K/V from pinned host memory and reads O back; the
     # copies of step i+1 run on their own streams while step i computes (device
@@ -431,6 +468,7 @@ def run_gpu(args):
                    "frac": round(append_bytes / (append_ms * 1e-3) / 1e9 /
                                  peaks["hbm_gbs"], 4)},
         "gpu_launches": K * 2,
+        "projection": proj,
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and spec.key == DEFAULT_WORKLOAD:

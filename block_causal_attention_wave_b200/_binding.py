@@ -67,6 +67,9 @@ _SIGS = {
                                                       ctypes.c_void_p, ctypes.c_void_p,
                                                       ctypes.c_void_p]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_qkv_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "wave_kv_append_batch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Node),
                                             ctypes.POINTER(ctypes.c_void_p),
                                             ctypes.POINTER(ctypes.c_void_p),
@@ -234,6 +237,14 @@ class KVCache:
         nt = (ctypes.c_int32 * max(n, 1))(*[K.shape[0] for K in Ks])
         _check(self.lib.wave_kv_append_batch(self.h, n, _nodes(entries), ks, vs, nt,
                                              _stream_handle(stream)))
+
+    def qkv_append(self, chunk, level, X, W, Q, stream=None):
+        """Project X [T][C] with W [3 H d][C] into Q (written to ``Q``, [T][H][d])
+        and the new entry's K/V pages, in one kernel."""
+        _check(self.lib.wave_qkv_append(self.h, chunk, level, ctypes.c_void_p(X.data_ptr()),
+                                        X.shape[0], X.shape[1], ctypes.c_void_p(W.data_ptr()),
+                                        ctypes.c_void_p(Q.data_ptr()), _stream_handle(stream)))
+        return Q
 
     def release(self, chunk, level):
         _check(self.lib.wave_kv_release(self.h, chunk, level))

@@ -44,6 +44,7 @@
 #include "exp2_poly.h"
 #include "ptx.cuh"
 #include "wave_internal.h"
+#include "wave_sync.cuh"
 
 using namespace wptx;
 
@@ -60,8 +61,6 @@ constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 softmax (2
 // thread; the host refuses to launch a build compiled with fewer.
 constexpr uint32_t kRegsLow = 88, kRegsHigh = 208, kRegsLaunch = 168;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
-constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr uint64_t kDrainNs = 200000000ull;
 constexpr uint32_t kPageMask = (1u << 25) - 1;  // page id bits of a page word
 constexpr int64_t kCounterOffset = 128;         // work-queue counter in the pool header
 
@@ -146,46 +145,6 @@ struct Bars {
                        COUNT = RING_EMPTY + kS;
   static_assert(COUNT * 8 + 16 + 4 * kItemSlots <= 448, "barrier area");  // 448..463: clock
 };
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// K-major operand (Q, K): rows of 128 bytes, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return smem_desc(addr, 16, 1024); }
-// MN-major operand (V as [key][d]): 64-column groups one panel (16 KB) apart,
-// 8-key groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_mn(uint32_t addr) { return smem_desc(addr, 16384, 1024); }
-
-struct Ctl {
-  volatile int* abort_flag;
-  int32_t* status;
-};
-
-// Bounded wait on an mbarrier phase. Returns false if this CTA is stopping.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& ctl, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if (*ctl.abort_flag) return false;
-    if ((++spins & 31u) == 0 && globaltimer_ns() - t0 > kTimeoutNs) {
-      *ctl.abort_flag = 1;
-      atomicCAS(ctl.status, 0, code);
-      return false;
-    }
-  }
-  return true;
-}
-
-// Bounded wait that ignores the stop flag: used only while stopping, to let
-// asynchronous copies or MMAs that were already issued complete.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kDrainNs) return;
-}
 
 struct Item {
   int node, head, pair;
@@ -604,20 +563,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     p.clock_out[0] = clock64() - clock_start[0];
     p.clock_out[1] = (int64_t)globaltimer_ns() - clock_start[1];
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
 }
 
 template <int D>

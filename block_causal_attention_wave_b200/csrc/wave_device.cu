@@ -11,6 +11,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "wave_internal.h"
 
@@ -90,6 +91,20 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
 static int cuda_fail(cudaError_t e, const char* what) {
   return fail(WAVE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
@@ -120,12 +135,8 @@ int device_init(wave_kv* kv) {
 
   // Tensor map over the page region: rows of head_dim bf16, box 64 x 128 with
   // the 128-byte swizzle the tensor-core shared-memory descriptors expect.
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
-    return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  auto encode = tensor_map_encoder();
+  if (!encode) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const int d = kv->cfg.head_dim, H = kv->cfg.heads;
   cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)kv->max_pages * 2 * H * kPageTokens};
   cuuint64_t strides[1] = {(cuuint64_t)d * 2};

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (type only; the driver is reached at run time)
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled (type only)
 
 #include <cstdint>
 #include <map>
@@ -57,6 +58,8 @@ int check_query_node(const wave_kv* kv, wave_node node);
 
 // Device halves (defined in .cu files).
 int device_init(wave_kv* kv);
+// The driver's tensor-map encoder, looked up once (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // One kernel launch copying the K/V of n entries (already allocated) into
 // their pages.
 int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,

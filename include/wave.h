@@ -134,6 +134,25 @@ int wave_kv_append_batch(wave_kv* kv, int32_t n_entries, const wave_node* entrie
                          const void* const* K, const void* const* V, const int32_t* ntokens,
                          void* stream);
 
+/* A node's QKV projection with its K/V append fused into the epilogue: one
+ * kernel computes [Q | K | V] = X W^T (fp32 accumulation, bf16 results) for
+ * the entry (chunk, level), writes Q to the caller's buffer, and writes K and
+ * V straight into the entry's new pages -- the same pages and bytes that
+ * wave_kv_alloc + wave_kv_append of those K and V would give. This is the
+ * producing side of the in-round K/V delivery of [WF] ("Key Findings"); the
+ * pages give no formula for the projection, so it is the plain linear map of
+ * a multi-head attention layer: no bias, no positional or norm term.
+ * X: device bf16 [ntokens][dim] (the node's hidden states), W: device bf16
+ * [3*H*d][dim] (a linear layer's [out][in] weight; output feature
+ * (s*H + h)*d + j is Q (s = 0), K (s = 1) or V (s = 2) of head h, component
+ * j), Q: device bf16 [ntokens][H][d], written. All caller-owned, contiguous,
+ * 16-byte aligned; dim a multiple of 64. Entry rules as wave_kv_alloc.
+ * Errors: as wave_kv_alloc, plus ARG (pointers, alignment, dim), CAPACITY
+ * (more than WAVE_MAX_APPEND_PAGES pages) and CUDA; on any error no pages stay
+ * taken. A device-side timeout is reported by wave_kv_status. */
+int wave_qkv_append(wave_kv* kv, int32_t chunk, int32_t level, const void* X, int32_t ntokens,
+                    int32_t dim, const void* W, void* Q, void* stream);
+
 /* Return the pages of (chunk, level) to the free set. Host only; the caller
  * must not release an entry that queued device work still reads (all library
  * kernels read the pool in stream order, so releasing after enqueueing the

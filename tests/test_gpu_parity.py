@@ -348,3 +348,68 @@ def test_append_batch_errors_take_nothing(cuda_lib):
         kv.append_batch([(1, 1), (0, 1)], [k, k], [k, k])
     assert e.value.code == -6 and kv.free_pages() == free0 - 1
     kv.status()
+
+
+def _qkv_case(wave, heads, head_dim, tokens, dim, rows=None):
+    """Fused projection + append of entry (1, 1) vs the oracle's X W^T."""
+    import torch
+    from oracle import projection
+    wl = wi.Workload("qkv", chunks=2, levels=1, heads=heads, head_dim=head_dim, tokens=tokens)
+    kv = make_cache(wave, wl, 2 * ((tokens + 127) // 128) + 4)
+    kv.alloc(0, 0)  # the entry's pages do not start at page 0
+    xb = wi.hidden_states(1, 1, tokens, dim)
+    wb = wi.qkv_weight(heads, head_dim, dim)
+    x, w = bits_to_torch(xb), bits_to_torch(wb)
+    q = torch.empty(tokens, heads, head_dim, dtype=torch.bfloat16, device="cuda")
+    kv.qkv_append(1, 1, x, w, q)
+    kv.status()
+    sel = np.arange(tokens) if rows is None else np.asarray(rows)
+    rq, rk, rv = projection.qkv(wi.bf16_bits_to_f64(xb[sel]), wi.bf16_bits_to_f64(wb), heads,
+                                head_dim)
+    assert_close(torch_to_f64(q)[sel], rq, "qkv Q", scale_with_output=True)
+    (table,) = kv.gather_table([(1, 1)], "clean")
+    own = table[-((tokens + 127) // 128):]
+    page_bytes, off, _ = kv.layout()
+    pool = kv.pool.cpu().numpy()
+    for kvi, ref in ((0, rk), (1, rv)):
+        got = np.zeros(((tokens + 127) // 128 * 128, heads, head_dim), dtype=np.uint16)
+        for pi, (page, valid) in enumerate(own):
+            base = off + page * page_bytes + kvi * heads * 128 * head_dim * 2
+            blk = pool[base:base + heads * 128 * head_dim * 2].view(np.uint16)
+            got[pi * 128:(pi + 1) * 128] = blk.reshape(heads, 128, head_dim).transpose(1, 0, 2)
+            assert valid == min(128, tokens - pi * 128)
+        assert not got[tokens:].any(), "page tail must be zero"
+        assert_close(wi.bf16_bits_to_f64(got[sel]), ref, f"qkv {'KV'[kvi]}",
+                     scale_with_output=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_qkv_append_small_ragged(cuda_lib, d):
+    """Three pages (300 tokens, ragged tail), three 64-wide slices of C."""
+    _qkv_case(cuda_lib, heads=3, head_dim=d, tokens=300, dim=192)
+
+
+def test_qkv_append_wan21_sampled_rows(cuda_lib):
+    """Wan2.1-1.3B shapes: 4680 tokens, C = 1536, 12 heads of 128; sampled rows
+    across every page, including the last (partial) one."""
+    rows = list(range(0, 4680, 37)) + [4607, 4608, 4679]
+    _qkv_case(cuda_lib, heads=12, head_dim=128, tokens=4680, dim=1536, rows=rows)
+
+
+def test_qkv_append_errors_take_nothing(cuda_lib):
+    import torch
+    wl = wi.Workload("qkv-err", chunks=2, levels=1, heads=2, head_dim=64, tokens=128)
+    kv = make_cache(cuda_lib, wl, 4)
+    free0 = kv.free_pages()
+    x = torch.zeros(128, 96, dtype=torch.bfloat16, device="cuda")  # C not a multiple of 64
+    w = torch.zeros(3 * 2 * 64, 96, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(128, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.qkv_append(0, 1, x, w, q)
+    assert e.value.code == -1 and kv.free_pages() == free0
+    x = torch.zeros(100, 64, dtype=torch.bfloat16, device="cuda")  # not tokens_per_chunk
+    w = torch.zeros(3 * 2 * 64, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cuda_lib.WaveError) as e:
+        kv.qkv_append(0, 1, x, w, q)
+    assert e.value.code == -1 and kv.free_pages() == free0
+    kv.status()

@@ -53,6 +53,20 @@ def normal_bf16(seed: int, shape, scale: float = 1.0) -> np.ndarray:
     return f32_to_bf16_bits(x)
 
 
+PROJ_SEED_BASE = SEED_BASE + 1_000_000  # projection inputs: disjoint from the ids above
+
+
+def hidden_states(chunk: int, level: int, tokens: int, dim: int) -> np.ndarray:
+    """``[tokens][dim]`` bf16 bits of N(0, 1): a node's hidden states (projection input)."""
+    return normal_bf16(PROJ_SEED_BASE + tensor_id("q", chunk, level), (tokens, dim))
+
+
+def qkv_weight(heads: int, head_dim: int, dim: int) -> np.ndarray:
+    """``[3 * heads * head_dim][dim]`` bf16 bits of N(0, 1) / sqrt(dim): a random
+    QKV projection weight in a linear layer's [out][in] layout."""
+    return normal_bf16(PROJ_SEED_BASE - 1, (3 * heads * head_dim, dim), 1.0 / math.sqrt(dim))
+
+
 def node_tensor(kind: str, chunk: int, level: int, tokens: int, heads: int,
                 head_dim: int, scale: float = 1.0) -> np.ndarray:
     """Token-major ``[tokens][heads][head_dim]`` bf16 bits for one (chunk, level)."""
