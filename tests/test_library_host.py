@@ -122,6 +122,11 @@ def test_error_paths(lib):
     with pytest.raises(wave.WaveError) as e:  # a host-only handle has no device to copy to
         kv.append_batch([(3, 1)], [k], [k], stream=0)
     assert e.value.code == -1 and kv.free_pages() == free
+    x = torch.zeros(200, 64, dtype=torch.bfloat16)
+    w = torch.zeros(3 * 2 * 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(wave.WaveError) as e:  # nor one to project on
+        kv.qkv_append(3, 1, x, w, k, stream=0)
+    assert e.value.code == -1 and kv.free_pages() == free
     with pytest.raises(wave.WaveError) as e:
         wave.KVCache(2, 96, 32, 2, pool=None, pool_bytes=1 << 20)
     assert e.value.code == -8
