@@ -368,7 +368,9 @@ def run_gpu(args):
         kv.status(stream)
         p_ms = pa.elapsed_time(pb) / (reps * len(active))
         p_flops = 2 * wl.tokens * 3 * wl.heads * wl.head_dim * dim
-        proj = {"kernel": "qkv_append_kernel", "what": "Q,K,V = X W^T per node, K/V written "
+        wide = wl.head_dim == 128 and (3 * wl.heads) % 2 == 0
+        proj = {"kernel": "qkv_append_wide_kernel" if wide else "qkv_append_kernel<%d>" % wl.head_dim,
+                "what": "Q,K,V = X W^T per node, K/V written "
                 "into the node's new pages in the epilogue", "dim": dim,
                 "flops_per_launch": p_flops, "avg_launch_ms": round(p_ms, 4),
                 "achieved": round(p_flops / (p_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",

@@ -383,10 +383,12 @@ def _qkv_case(wave, heads, head_dim, tokens, dim, rows=None):
                      scale_with_output=True)
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_qkv_append_small_ragged(cuda_lib, d):
-    """Three pages (300 tokens, ragged tail), three 64-wide slices of C."""
-    _qkv_case(cuda_lib, heads=3, head_dim=d, tokens=300, dim=192)
+@pytest.mark.parametrize("heads,d", [(3, 64), (3, 128), (2, 128)])
+def test_qkv_append_small_ragged(cuda_lib, heads, d):
+    """Three pages (300 tokens, ragged tail), three 64-wide slices of C. With d
+    128 and 3 H even the 256-feature persistent kernel runs (H = 2), else the
+    128-feature one."""
+    _qkv_case(cuda_lib, heads=heads, head_dim=d, tokens=300, dim=192)
 
 
 def test_qkv_append_wan21_sampled_rows(cuda_lib):
