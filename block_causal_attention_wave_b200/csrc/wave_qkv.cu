@@ -10,8 +10,10 @@
 // producing side of the in-round K/V delivery of the Wave Forcing page ("Key
 // Findings"): the K/V reach the round's cache without a separate copy.
 //
-// How: one CTA per output tile of 128 tokens x one head's d features of Q, K
-// or V -- for K and V exactly one page tile. 128 threads:
+// How (two kernels). With d = 128 and 3 H even, qkv_append_wide_kernel (below)
+// takes tiles of 128 tokens x 256 features in persistent CTAs. Otherwise one
+// CTA per output tile of 128 tokens x one head's d features of Q, K or V --
+// for K and V exactly one page tile. 128 threads:
 //   warp 0 lane 0  TMA producer: 64-column slices of the X tile and the W tile
 //                  (both K-major, 128-byte swizzle) into a 3-stage ring;
 //   warp 1 lane 0  tcgen05 issuer: four M128 x Nd x K16 MMAs per slice into
