@@ -8,23 +8,23 @@
 // over the tokens of the node's key list (prefix, history E(c-r, phi(l, r)),
 // own E(c, l)) -- full attention inside every listed chunk, nothing else.
 //
-// How (B200 design, not the pages'): one CTA per SM, each looping over work
-// items (node, head, 128-query tile) ordered longest key list first, query
-// tiles of one head adjacent so concurrent CTAs share that head's K/V pages in
-// L2. Per CTA:
-//   warp 0   TMA producer: Q tile once per item, then each 128-token K and V
-//            page of the key list, gathered by page id (the page id is the
-//            tensor-map row coordinate), into a 3-stage shared-memory ring.
-//   warp 1   tcgen05 issuer: S = Q K^T (both operands in shared memory,
-//            128-byte swizzle, K-major) into one of two TMEM S buffers, then
-//            O += P V with P read from TMEM (bf16) and V from shared memory
-//            (MN-major). O accumulates in TMEM in fp32.
-//   warps 2-5  softmax: one query row per thread. tcgen05.ld of the S row,
-//            padding keys of a partial page masked, online max in the log2
-//            domain, exp2, bf16 P written back to TMEM with tcgen05.st. O is
-//            rescaled only when the running max grows by more than 8 (log2
-//            units); otherwise the stale max is kept, which is exact after the
-//            final division because P <= 2^8 stays well inside fp32/bf16 range.
+// How (B200 design, not the pages'): one CTA per SM, each claiming work items
+// (node, head, pair of 128-query tiles) longest key list first from a global
+// counter; query tiles of one head are adjacent, so concurrent CTAs share that
+// head's K/V pages in L2. Per CTA (384 threads):
+//   warp 0   TMA producer: both Q tiles once per item, then each 128-token K
+//            and V page of the key list, gathered by page id (the tensor-map
+//            row coordinate), into a 5-slot (d = 64: 10-slot) shared ring.
+//   warp 1   tcgen05 issuer: S_w = Q_w K^T (both operands in shared memory,
+//            128-byte swizzle, K-major) into TMEM S buffer w, then O_w += P_w V
+//            with P_w read from TMEM (bf16, inside S_w) and V from shared
+//            memory (MN-major); the two query tiles ping-pong on the pipe.
+//   warps 4-11  softmax, one warpgroup per query tile, one row per thread:
+//            tcgen05.ld of the S row, padding keys of a partial page masked,
+//            max in the log2 domain, exp2, bf16 P written back with
+//            tcgen05.st. O is rescaled only when the running max grows by
+//            more than 8 (log2 units); otherwise the stale max is kept, exact
+//            after the final division as P <= 2^8 stays inside fp32/bf16.
 //            Epilogue: O / l, bf16, stored straight from registers (only rows
 //            that belong to the node).
 // Every wait is bounded (2 s); on timeout the kernel records a status word,
