@@ -139,3 +139,26 @@ def test_error_paths(lib):
     with pytest.raises(wave.WaveError) as e:
         kv.round_attn([(0, 2)], "progressive", q, q, stream=0)
     assert e.value.code == -1
+
+
+def test_random_rollouts_match_oracle_bit_exact(lib):
+    """Seeded random shapes (chunks, levels, window, tokens incl. ragged and
+    exact multiples of 128, prefix, policy): schedules, last-read tables and
+    every round's gather table equal the oracle's."""
+    import numpy as np
+    rng = np.random.default_rng(20261202)
+    for case in range(150):
+        B = int(rng.integers(1, 10))
+        K = int(rng.integers(1, 6))
+        W = int(rng.choice([0, 1, 2, 3, 5]))
+        T = int(rng.choice([1, 64, 127, 128, 129, 300, 1000]))
+        prefix = int(rng.choice([0, 0, 1, 128, 200]))
+        pol = str(rng.choice(wi.POLICIES))
+        wl = wi.Workload(f"rand{case}", chunks=B, levels=K, heads=1, head_dim=64, tokens=T,
+                         window=W, prefix=prefix)
+        assert wave.schedule(B, K, pol, W) == osched.schedule(B, K, pol, W), (B, K, W, pol)
+        assert wave.last_read_rounds(B, K, pol, W) == osched.last_read_round(B, K, pol, W)
+        max_pages = 2000
+        got = _library_rollout(wl, pol, max_pages)
+        want = ocache.rollout_tables(B, K, pol, W, T, prefix, max_pages)
+        assert got == [(a, t) for a, t in want], (B, K, W, T, prefix, pol)
