@@ -52,3 +52,16 @@ def test_reduce_max_over_two_gloo_ranks():
 def test_reduce_max_without_process_group_is_identity():
     import bench
     assert bench.reduce_max(3.5) == 3.5
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun the oracle arm prints from rank 0 alone; other ranks exit
+    without work (and without a process group of their own)."""
+    import argparse
+
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.run_reference(argparse.Namespace(steps=1, warmup=3)) is None
+    assert capsys.readouterr().out == ""
