@@ -67,6 +67,7 @@ _SIGS = {
                                                       ctypes.c_void_p, ctypes.c_void_p,
                                                       ctypes.c_void_p]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_kv_set_wait_limit": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64]),
     "wave_qkv_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
@@ -289,6 +290,10 @@ class KVCache:
     def status(self, stream=None):
         """Synchronise and raise WaveError if a kernel timed out."""
         _check(self.lib.wave_kv_status(self.h, _stream_handle(stream)))
+
+    def set_wait_limit(self, ns: int = 0):
+        """Bound on one device wait of later launches (ns; 0 = default 2 s)."""
+        _check(self.lib.wave_kv_set_wait_limit(self.h, int(ns)))
 
     def last_launch_clock(self, stream=None):
         """(SM cycles, nanoseconds) of the last attention launch's first CTA;

@@ -15,18 +15,21 @@
 //   warp 0   TMA producer: both Q tiles once per item, then each 128-token K
 //            and V page of the key list, gathered by page id (the tensor-map
 //            row coordinate), into a 5-slot (d = 64: 10-slot) shared ring.
-//   warp 1   tcgen05 issuer: S_w = Q_w K^T (both operands in shared memory,
-//            128-byte swizzle, K-major) into TMEM S buffer w, then O_w += P_w V
-//            with P_w read from TMEM (bf16, inside S_w) and V from shared
-//            memory (MN-major); the two query tiles ping-pong on the pipe.
+//   warp 1   tcgen05 issuer: S = Q_w K^T (both operands in shared memory,
+//            128-byte swizzle, K-major) into the one TMEM S buffer, then
+//            O_w += P_w V with P_w read from TMEM (bf16, its own 64 columns)
+//            and V from shared memory (MN-major). Pipe order per page t:
+//            S_0(t), PV_0(t-1), S_1(t), PV_1(t-1): the S buffer is reloaded
+//            while the P.V behind it runs, and a tile's P(t) is needed only
+//            after the next page's S, a whole page period after its S(t).
 //   warps 4-11  softmax, one warpgroup per query tile, one row per thread:
-//            tcgen05.ld of the S row, padding keys of a partial page masked,
-//            max in the log2 domain, exp2, bf16 P written back with
-//            tcgen05.st. O is rescaled only when the running max grows by
-//            more than 8 (log2 units); otherwise the stale max is kept, exact
-//            after the final division as P <= 2^8 stays inside fp32/bf16.
-//            Epilogue: O / l, bf16, stored straight from registers (only rows
-//            that belong to the node).
+//            tcgen05.ld of the S row (then S is handed back), padding keys of
+//            a partial page masked, max in the log2 domain, exp2, bf16 P
+//            written to P_w with tcgen05.st. O is rescaled only when the
+//            running max grows by more than 8 (log2 units); otherwise the
+//            stale max is kept, exact after the final division as P <= 2^8
+//            stays inside fp32/bf16. Epilogue: O / l, bf16, stored straight
+//            from registers (only rows that belong to the node).
 // Every wait is bounded (2 s); on timeout the kernel records a status word,
 // every role stops, and TMEM is freed before exit.
 #include <cuda.h>
@@ -56,10 +59,17 @@ constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 softmax (2
 // Register split after start-up (setmaxnreg): warps 0..3 (TMA, MMA, two idle;
 // one per SM sub-partition) drop to kRegsLow, the two softmax warpgroups (two
 // warps per sub-partition) rise to kRegsHigh, so each softmax thread can hold
-// a full 128-column S row. Per sub-partition 88 + 2 x 208 = 504 <= 512
-// registers per lane, i.e. the sum equals what the launch holds at 168 per
-// thread; the host refuses to launch a build compiled with fewer.
-constexpr uint32_t kRegsLow = 88, kRegsHigh = 208, kRegsLaunch = 168;
+// a full 128-column S row without spilling. Per sub-partition
+// kRegsLow + 2 kRegsHigh <= 504 registers per lane, i.e. at most what the
+// launch holds at 168 per thread; the host refuses to launch a build compiled
+// with fewer.
+#ifndef WAVE_REGS_LOW
+#define WAVE_REGS_LOW 72
+#endif
+#ifndef WAVE_REGS_HIGH
+#define WAVE_REGS_HIGH 216
+#endif
+constexpr uint32_t kRegsLow = WAVE_REGS_LOW, kRegsHigh = WAVE_REGS_HIGH, kRegsLaunch = 168;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kPageMask = (1u << 25) - 1;  // page id bits of a page word
 constexpr int64_t kCounterOffset = 128;         // work-queue counter in the pool header
@@ -80,6 +90,7 @@ struct AttnParams {
   int32_t* status;    // device status word (pool header)
   int32_t* counter;   // work-queue counter, zero at launch (pool header)
   int64_t* clock_out; // CTA 0's SM cycles and nanoseconds (pool header)
+  uint64_t wait_ns;   // bound on one barrier wait
   float scale_log2;   // log2(e) / sqrt(d)
   int32_t heads;
   int32_t n_nodes;
@@ -113,9 +124,12 @@ struct Cfg {
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
-  // TMEM columns: S_w at 128 w (fp32; P_w as bf16x2 overwrites its first 64
-  // columns), O_w at 256 + 128 w.
-  static constexpr uint32_t kColS = 0, kColO = 256, kCols = 512;
+  // TMEM columns: one S buffer (fp32, 128 keys) that the two query tiles
+  // take in turn, P_w (bf16x2, 64 columns) at 128 + 64 w, O_w at 256 + 128 w.
+  // S is free again as soon as its softmax warpgroup has loaded it, so the next
+  // S = Q K^T need not wait for the previous P.V: the softmax of a tile has a
+  // whole page period of MMAs (both tiles' S and P.V) to hide in.
+  static constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kCols = 512;
   // Instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128.
   static constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
                                       ((128u >> 4) << 24);
@@ -127,10 +141,12 @@ struct Cfg {
 enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
-  B_S_FULL,                 // 2: S_w computed
-  B_P_FULL = B_S_FULL + 2,  // 2: P_w written (128 arrivals)
-  B_O_FULL = B_P_FULL + 2,  // 2: last P.V of an item done
-  B_O_EMPTY = B_O_FULL + 2, // 2: epilogue has read O_w (128 arrivals)
+  B_S_FULL,                  // 2: S = Q_w K^T computed into the S buffer
+  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (128 arrivals)
+  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (128 arrivals)
+  B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
+  B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
+  B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
   B_DRAIN = B_O_EMPTY + 2,
   B_ITEM_FULL,              // 2: next work item published by the producer
   B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by the MMA thread and 8 softmax warps
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * BR::COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 4);
   volatile int* item_q = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 8);
-  const Ctl ctl{abort_flag, p.status};
+  const Ctl ctl{abort_flag, p.status, p.wait_ns};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -215,7 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_Q_EMPTY), 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(B_S_FULL + w), 1);
+      mbar_init(bar(B_S_FREE + w), 128);
       mbar_init(bar(B_P_FULL + w), 128);
+      mbar_init(bar(B_P_FREE + w), 1);
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
     }
@@ -315,8 +333,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ---------------------------------------------------------- tcgen05 issuer
       if (lane == 0) {
-        // g: K/V tiles consumed; gw/itw: tiles/items processed by query tile w.
-        uint32_t g = 0, it = 0, gw[2] = {0, 0}, itw[2] = {0, 0};
+        // g: pages consumed; pv[w]: P.V MMAs issued for query tile w (= P_w
+        // buffers consumed); sc[w]: S MMAs issued for tile w; itw[w]: items
+        // done by tile w; s_last: tile whose S the buffer holds (-1: none).
+        uint32_t g = 0, it = 0, pv[2] = {0, 0}, sc[2] = {0, 0}, itw[2] = {0, 0};
+        int s_last = -1;
         bool ok = true;
         auto ring_wait = [&](uint32_t r, int code) -> bool {
           return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
@@ -330,29 +351,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
         auto lo_k = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | (1u << 16); };
         auto lo_mn = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | ((16384u >> 4) << 16); };
-        // S_w = Q_w K(t)^T into TMEM columns 128 w.
-        auto issue_s = [&](int w, uint32_t t) {
+        // S = Q_w K(t)^T into the S buffer, once the softmax warpgroup that
+        // owns the buffer's previous contents has loaded them.
+        auto issue_s = [&](int w, uint32_t t) -> bool {
+          if (s_last >= 0 &&
+              !wait_bar(bar(B_S_FREE + s_last), (sc[s_last] - 1) & 1, ctl, 0x119 + s_last))
+            return false;
+          tc_fence_after();
           const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
           const uint32_t kaddr = slot_addr(2 * t);
           if constexpr (D == 128) {
             mma_ss_k128<2, C::kPanelBytes / 16, 2, C::kPanelBytes / 16>(
-                tmem + C::kColS + 128 * w, lo_k(qaddr), kDescHi, lo_k(kaddr), kDescHi, C::kIdescS,
-                0u);
+                tmem + C::kColS, lo_k(qaddr), kDescHi, lo_k(kaddr), kDescHi, C::kIdescS, 0u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-              mma_ss(tmem + C::kColS + 128 * w, desc_k(qaddr + off), desc_k(kaddr + off),
-                     C::kIdescS, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + C::kColS, desc_k(qaddr + off), desc_k(kaddr + off), C::kIdescS,
+                     kk > 0 ? 1u : 0u);
             }
           }
+          tc_commit(bar(B_S_FULL + w));
+          ++sc[w];
+          s_last = w;
+          return true;
         };
-        // O_w (+)= P_w V(t), P_w read from TMEM (bf16 in S_w's first 64 columns).
-        auto issue_pv = [&](int w, uint32_t t, bool accumulate) {
+        // O_w (+)= P_w V(t), P_w read from TMEM, once softmax w has written P_w
+        // (and, for an item's first P.V, once its epilogue has read O_w). The
+        // commit on P_FREE_w lets softmax w overwrite P_w (and touch O_w).
+        auto issue_pv = [&](int w, uint32_t t, bool accumulate, bool v_wait) -> bool {
+          if (!wait_bar(bar(B_P_FULL + w), pv[w] & 1, ctl, 0x112 + w)) return false;
+          if (!accumulate && itw[w] > 0 &&
+              !wait_bar(bar(B_O_EMPTY + w), (itw[w] - 1) & 1, ctl, 0x114 + w))
+            return false;
+          if (v_wait && !ring_wait(2 * t + 1, 0x116)) return false;
+          tc_fence_after();
           const uint32_t vaddr = slot_addr(2 * t + 1);
-          mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * w, tmem + C::kColS + 128 * w,
+          mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * w, tmem + C::kColP + 64 * w,
                                  lo_mn(vaddr), kDescHi, C::kIdescO, accumulate ? 1u : 0u);
+          tc_commit(bar(B_P_FREE + w));
+          ++pv[w];
+          return true;
         };
+        // Pipe order per page t: S_0(t), PV_0(t-1), S_1(t), PV_1(t-1). A
+        // tile's P(t) is consumed after S of page t+1, so its softmax has the
+        // three other MMA groups in between; the S buffer is reloaded while
+        // the P.V behind it runs.
         for (uint32_t k = 0; ok; ++k) {
           int item;
           if (!next_item(k, 0x118, item)) { ok = false; break; }
@@ -362,43 +406,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = p.nodes[w.node].n_pages;
           const int nq = w.two ? 2 : 1;
           if (!wait_bar(bar(B_Q_FULL), it & 1, ctl, 0x110)) { ok = false; break; }
-          if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
-          tc_fence_after();
-          for (int q = 0; q < nq; ++q) {
-            issue_s(q, g);
-            tc_commit(bar(B_S_FULL + q));
-          }
-          tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));
-          if (n == 1) tc_commit(bar(B_Q_EMPTY));
-          for (int j = 0; j < n; ++j, ++g) {
-            const bool more = j + 1 < n;
+          for (int j = 0; j < n && ok; ++j, ++g) {
+            if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
             for (int q = 0; q < nq; ++q) {
-              if (!wait_bar(bar(B_P_FULL + q), gw[q] & 1, ctl, 0x112 + q)) { ok = false; break; }
-              if (j == 0 && itw[q] > 0 &&
-                  !wait_bar(bar(B_O_EMPTY + q), (itw[q] - 1) & 1, ctl, 0x114 + q)) {
-                ok = false;
-                break;
+              if (!issue_s(q, g)) { ok = false; break; }
+              if (q == nq - 1) {
+                tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));  // K(g) done
+                if (j == n - 1) tc_commit(bar(B_Q_EMPTY));
               }
-              if (q == 0 && !ring_wait(2 * g + 1, 0x116)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv(q, g, j > 0);
-              ++gw[q];
-              if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * g + 1) % S));  // V(g) done
-              if (more) {
-                if (q == 0 && !ring_wait(2 * g + 2, 0x117)) { ok = false; break; }
-                tc_fence_after();
-                issue_s(q, g + 1);
-                tc_commit(bar(B_S_FULL + q));
-                if (q == nq - 1) {
-                  tc_commit(bar(BR::RING_EMPTY + (2 * g + 2) % S));  // K(g+1) done
-                  if (j + 2 == n) tc_commit(bar(B_Q_EMPTY));
-                }
-              } else {
-                tc_commit(bar(B_O_FULL + q));
+              if (j > 0) {
+                if (!issue_pv(q, g - 1, j > 1, q == 0)) { ok = false; break; }
+                if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * (g - 1) + 1) % S));
               }
             }
-            if (!ok) break;
           }
+          if (!ok) break;
+          // The item's last page: P.V of both tiles, then O is complete.
+          for (int q = 0; q < nq; ++q) {
+            if (!issue_pv(q, g - 1, n > 1, q == 0)) { ok = false; break; }
+            tc_commit(bar(B_O_FULL + q));
+            if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * (g - 1) + 1) % S));
+          }
+          if (!ok) break;
           for (int q = 0; q < nq; ++q) ++itw[q];
           ++it;
         }
@@ -414,10 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;    // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t tS = trow + C::kColS + 128 * wq;
+    const uint32_t tS = trow + C::kColS;
+    const uint32_t tP = trow + C::kColP + 64 * wq;
     const uint32_t tO = trow + C::kColO + 128 * wq;
     const float sl2 = p.scale_log2;
-    uint32_t g = 0, it = 0;  // tiles and items processed by this warpgroup
+    // g: S tiles loaded, pw: P_w written (each one read by a P.V that commits
+    // P_FREE_w), it: items finished by this warpgroup.
+    uint32_t g = 0, pw = 0, it = 0;
     for (uint32_t k = 0;; ++k) {
       int item;
       bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, item));
@@ -434,12 +466,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int valid = (int)(p.pages[nd.page0 + t] >> 25) + 1;
-        // The whole S row in one TMEM round trip.
+        // The whole S row in one TMEM round trip; then the S buffer goes back
+        // to the MMA thread for the other tile's (or the next page's) S.
         float sv[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_S_FREE + wq));
         if (valid < 128) {  // partial last page of an entry: drop the padding keys
 #pragma unroll
           for (int i = 0; i < 128; ++i) sv[i] = i < valid ? sv[i] : -INFINITY;
@@ -457,11 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  fmaxf(mx[6], mx[7]));
         const float m_new = fmaxf(m_run, mrow * sl2);
         const bool grow = __any_sync(0xffffffffu, t > 0 && m_new > m_run + 8.f);
+        // P_w and O_w are ours again once the P.V that read the previous P_w
+        // has finished (it was issued right after this page's S).
+        bool p_free = pw == 0;
         if (t == 0) {
           m_run = m_new;
         } else if (grow) {
-          // Bring O up to the new max. The P.V of the previous tile is done:
-          // it was issued before this tile's S, whose completion we waited for.
+          ok = __all_sync(0xffffffffu, wait_bar(bar(B_P_FREE + wq), (pw - 1) & 1, ctl, 0x126 + wq));
+          if (!ok) break;
+          tc_fence_after();
+          p_free = true;
+          // Bring O up to the new max (O holds every P.V up to the previous page).
           const float alpha = ex2_approx(m_run - m_new);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -475,7 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run *= alpha;
           m_run = m_new;
         }
-        // P = 2^(S log2e/sqrt(d) - m), packed to bf16 into S's first 64 columns.
+        // P = 2^(S log2e/sqrt(d) - m), packed to bf16 in registers, then stored
+        // to P_w in two 32-column pieces.
         const float negm = -m_run;
 #if WAVE_PACKED_FMA
         const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(negm, negm);
@@ -484,20 +526,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #endif
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 16 columns of S -> 8 columns of P
-          uint32_t pk[8];
+        for (int h = 0; h < 2; ++h) {  // 64 columns of S -> 32 columns of P
+          uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < 32; ++i) {
+            const int c = 64 * h + 2 * i;
             float x0, x1;
 #if WAVE_PACKED_FMA
-            f2_unpack(f2_fma(f2_pack(sv[c * 16 + 2 * i], sv[c * 16 + 2 * i + 1]), scale2, negm2), x0,
-                      x1);
+            f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), scale2, negm2), x0, x1);
 #else
-            x0 = fmaf(sv[c * 16 + 2 * i], sl2, negm);
-            x1 = fmaf(sv[c * 16 + 2 * i + 1], sl2, negm);
+            x0 = fmaf(sv[c], sl2, negm);
+            x1 = fmaf(sv[c + 1], sl2, negm);
 #endif
             float y0, y1;
-            if (((c & 1) * 16 + 2 * i) < kEmuPerChunk) {
+            if ((c & 31) < kEmuPerChunk) {
               exp2_poly2(x0, x1, y0, y1);
             } else {
               y0 = ex2_approx(x0);
@@ -510,8 +552,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #endif
             pk[i] = pack_bf16x2(y0, y1);
           }
-          tmem_st8(tS + c * 8, pk);
+          if (h == 0 && !p_free) {
+            ok = __all_sync(0xffffffffu,
+                            wait_bar(bar(B_P_FREE + wq), (pw - 1) & 1, ctl, 0x126 + wq));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          tmem_st32(tP + 32 * h, pk);
         }
+        if (!ok) break;
 #if WAVE_PACKED_FMA
         float acc[4];
         f2_unpack(acc2[0], acc[0], acc[1]);
@@ -521,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL + wq));
+        ++pw;
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, wait_bar(bar(B_O_FULL + wq), it & 1, ctl, 0x122 + wq));
@@ -605,6 +655,7 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
                     const void* Q, void* O, void* stream, int32_t* counter) {
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
+  if (int rc = check_current_device(kv)) return rc;
   if (!valid_policy(policy)) return fail(WAVE_ERR_ARG, "unknown policy %d", policy);
   if (n_active < 0 || (n_active > 0 && !active)) return fail(WAVE_ERR_ARG, "bad active list");
   if (n_active == 0) return WAVE_OK;
@@ -640,6 +691,7 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
   prm.counter = counter;
   prm.clock_out = reinterpret_cast<int64_t*>(static_cast<char*>(kv->cfg.pool) + 256);
+  prm.wait_ns = wait_limit_ns(kv);
   prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   prm.heads = H;
   prm.q_rows = T;

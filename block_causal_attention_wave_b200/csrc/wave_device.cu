@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "wave_internal.h"
+#include "wave_sync.cuh"
 
 namespace wavei {
 
@@ -149,6 +150,17 @@ int device_init(wave_kv* kv) {
   if (r != CUDA_SUCCESS) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled(pool) failed: %d", (int)r);
   return WAVE_OK;
 }
+
+int check_current_device(const wave_kv* kv) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != kv->device)
+    return fail(WAVE_ERR_ARG, "current device %d is not the pool's device %d", dev, kv->device);
+  return WAVE_OK;
+}
+
+uint64_t wait_limit_ns(const wave_kv* kv) { return kv->wait_ns ? kv->wait_ns : kTimeoutNs; }
 
 int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,
                   const void* const* K, const void* const* V, void* stream) {

@@ -217,6 +217,13 @@ int wave_kv_release(wave_kv* kv, int32_t chunk, int32_t level) {
   return WAVE_OK;
 }
 
+int wave_kv_set_wait_limit(wave_kv* kv, uint64_t ns) {
+  clear_error();
+  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+  kv->wait_ns = ns;
+  return WAVE_OK;
+}
+
 int wave_kv_free_pages(const wave_kv* kv, int32_t* n) {
   clear_error();
   if (!kv || !n) return fail(WAVE_ERR_ARG, "NULL argument");
@@ -236,6 +243,7 @@ int wave_kv_append_batch(wave_kv* kv, int32_t n_entries, const wave_node* entrie
   clear_error();
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL) cannot append");
+  if (int rc = check_current_device(kv)) return rc;
   if (n_entries < 0 || (n_entries > 0 && (!entries || !K || !V || !ntokens)))
     return fail(WAVE_ERR_ARG, "bad arguments");
   if (n_entries > WAVE_MAX_APPEND_ENTRIES)

@@ -28,6 +28,7 @@ struct wave_kv {
   bool on_device = false;  // pool != NULL
   int device = -1;
   int num_sms = 0;
+  uint64_t wait_ns = 0;     // bound on one device wait; 0 = the default (2 s)
   alignas(64) CUtensorMap tm_kv;  // rows of d bf16 over every page's K and V
 };
 
@@ -58,6 +59,11 @@ int check_query_node(const wave_kv* kv, wave_node node);
 
 // Device halves (defined in .cu files).
 int device_init(wave_kv* kv);
+// WAVE_ERR_ARG unless the calling thread's current device is the pool's: the
+// handle's tensor maps and pool pointer belong to that device.
+int check_current_device(const wave_kv* kv);
+// The handle's bound on one device wait, in nanoseconds.
+uint64_t wait_limit_ns(const wave_kv* kv);
 // The driver's tensor-map encoder, looked up once (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // One kernel launch copying the K/V of n entries (already allocated) into

@@ -68,6 +68,7 @@ struct QkvParams {
   uint8_t* data;        // pool + data_offset
   int64_t page_bytes;
   int32_t* status;      // device status word (pool header)
+  uint64_t wait_ns;     // bound on one barrier wait
   int32_t ntokens;
   int32_t heads;
   int32_t k_slices;     // C / 64
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(kQkvThreads, 2) qkv_append_kernel(const __grid
   auto bar = [&](int i) -> uint32_t { return sb + C::kBarOff + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * C::kBars + 4);
-  const Ctl ctl{abort_flag, p.status};
+  const Ctl ctl{abort_flag, p.status, p.wait_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tile = blockIdx.x;          // 128-token tile = page of the entry
   const int which = blockIdx.y / p.heads;  // 0 Q, 1 K, 2 V
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sb + C::kBarOff + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * C::kBars + 4);
-  const Ctl ctl{abort_flag, p.status};
+  const Ctl ctl{abort_flag, p.status, p.wait_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = p.k_slices, n_tiles = p.n_tiles, n_m = p.n_mtiles;
 
@@ -430,6 +431,7 @@ int qkv_append_impl(wave_kv* kv, const wave_entry& ent, const void* X, int32_t d
   prm.data = static_cast<uint8_t*>(kv->cfg.pool) + kv->data_offset;
   prm.page_bytes = kv->page_bytes;
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
+  prm.wait_ns = wait_limit_ns(kv);
   prm.ntokens = ent.ntokens;
   prm.heads = H;
   prm.k_slices = dim / 64;
@@ -456,6 +458,7 @@ extern "C" int wave_qkv_append(wave_kv* kv, int32_t chunk, int32_t level, const 
   clear_error();
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL) cannot append");
+  if (int rc = check_current_device(kv)) return rc;
   if (!X || !W || !Q ||
       ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(Q)) & 15))
     return fail(WAVE_ERR_ARG, "X, W and Q must be non-NULL and 16-byte aligned");

@@ -25,6 +25,9 @@
  *   - Device buffers are caller-owned. The library never calls cudaMalloc; the
  *     K/V pool is one caller-provided device buffer (see wave_kv_config).
  *   - Activations are bf16, token-major and contiguous: [tokens][heads][head_dim].
+ *   - Calls that launch kernels (append, projection, attention) must be made
+ *     with the pool's device current (the device current at wave_kv_create);
+ *     otherwise they return WAVE_ERR_ARG before taking pages or launching.
  *   - No call is thread-safe on the same wave_kv handle.
  */
 #ifndef WAVE_H_
@@ -218,6 +221,16 @@ int wave_round_attn_static_scratch(wave_kv* kv, const wave_node* active, int32_t
  * the driver every few milliseconds miss short clock reductions. Both are 0
  * before the first launch and for a host-only handle. Errors: ARG, CUDA. */
 int wave_kv_last_launch_clock(wave_kv* kv, void* stream, int64_t* cycles, int64_t* ns);
+
+/* Bound on how long one wait inside a kernel launched on this handle may take
+ * (attention and fused projection; the append kernel does not wait), in
+ * nanoseconds; 0 restores the default of 2 s. A wait that runs out makes the
+ * kernel stop every role, finish the copies and MMAs it has issued, free its
+ * tensor memory and return; the launch's output is then undefined and the
+ * next wave_kv_status reports WAVE_ERR_TIMEOUT. This is the failure-detection
+ * path: a small bound lets a test make a wait run out without faulting the
+ * GPU. Applies to launches made after the call. Host only. Errors: ARG. */
+int wave_kv_set_wait_limit(wave_kv* kv, uint64_t ns);
 
 /* Synchronise `stream`, then read and clear the pool's device status word.
  * Returns WAVE_OK, WAVE_ERR_TIMEOUT if a kernel gave up on a bounded wait
