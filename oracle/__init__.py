@@ -20,6 +20,11 @@ What it computes, each part written as the plain definition from the pages:
                                earlier, cleaner chunks).
 * ``projection``            -- a node's Q, K, V = X W^T split by (Q/K/V, head),
                                in float64 (the K/V of in-round delivery).
+* ``block``                 -- the rest of one transformer block of a round:
+                               rotary position embedding of Q and K over
+                               (frame, row, column), out-projection and
+                               tanh-GELU MLP with residuals, bf16 storage
+                               between kernels (readings stated there).
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
 against something other than itself (brute-force dense masks, closed forms,
@@ -27,4 +32,4 @@ torch's CPU attention, exhaustive search). Absolute attention values printed by
 the pages: none exist, so that part is "parity unpinned" against the pages and
 pinned only by the mathematics.
 """
-from . import policy, schedule, cache, attention, projection  # noqa: F401
+from . import policy, schedule, cache, attention, projection, block  # noqa: F401
