@@ -15,13 +15,14 @@
 //   warp 0   TMA producer: both Q tiles once per item, then each 128-token K
 //            and V page of the key list, gathered by page id (the tensor-map
 //            row coordinate), into a 5-slot (d = 64: 10-slot) shared ring.
-//   warp 1   tcgen05 issuer: S = Q_w K^T (both operands in shared memory,
-//            128-byte swizzle, K-major) into the one TMEM S buffer, then
-//            O_w += P_w V with P_w read from TMEM (bf16, its own 64 columns)
-//            and V from shared memory (MN-major). Pipe order per page t:
-//            S_0(t), PV_0(t-1), S_1(t), PV_1(t-1): the S buffer is reloaded
-//            while the P.V behind it runs, and a tile's P(t) is needed only
-//            after the next page's S, a whole page period after its S(t).
+//   warps 1, 3  tcgen05 issuers, one per query tile w: S = Q_w K^T (both
+//            operands in shared memory, 128-byte swizzle, K-major) into the
+//            one TMEM S buffer, then O_w += P_w V with P_w read from TMEM
+//            (bf16, its own 64 columns) and V from shared memory (MN-major).
+//            Pipe order per page t: S_0(t), PV_0(t-1), S_1(t), PV_1(t-1): the
+//            S buffer is reloaded while the P.V behind it runs, and a tile's
+//            P(t) is needed only after the next page's S. Two issuing threads
+//            keep the tensor pipe's short queue fed while either one waits.
 //   warps 4-11  softmax, one warpgroup per query tile, one row per thread:
 //            tcgen05.ld of the S row (then S is handed back), padding keys of
 //            a partial page masked, max in the log2 domain, exp2, bf16 P
@@ -55,7 +56,7 @@ namespace wavei {
 
 namespace {
 
-constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 softmax (2 groups)
+constexpr int kThreads = 384;  // warp 0 TMA, warps 1 and 3 MMA, warps 4..11 softmax (2 groups)
 // Register split after start-up (setmaxnreg): warps 0..3 (TMA, MMA, two idle;
 // one per SM sub-partition) drop to kRegsLow, the two softmax warpgroups (two
 // warps per sub-partition) rise to kRegsHigh, so each softmax thread can hold
@@ -147,9 +148,9 @@ enum : int {
   B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
   B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
-  B_DRAIN = B_O_EMPTY + 2,
-  B_ITEM_FULL,              // 2: next work item published by the producer
-  B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by the MMA thread and 8 softmax warps
+  B_DRAIN = B_O_EMPTY + 2,   // 2: every MMA of MMA thread w done (while stopping)
+  B_ITEM_FULL = B_DRAIN + 2, // 2: next work item published by the producer
+  B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by the 2 MMA threads and 8 softmax warps
   B_RING_FULL = B_ITEM_EMPTY + 2,  // kSlots each from here
 };
 constexpr int kItemSlots = 2;
@@ -239,12 +240,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < kItemSlots; ++k) {
       mbar_init(bar(B_ITEM_FULL + k), 1);
-      mbar_init(bar(B_ITEM_EMPTY + k), 1 + 8);  // MMA thread + one lane per softmax warp
+      mbar_init(bar(B_ITEM_EMPTY + k), 2 + 8);  // MMA threads + one lane per softmax warp
     }
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_DRAIN + 1), 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(BR::RING_FULL + s), 1);
-      mbar_init(bar(BR::RING_EMPTY + s), 1);
+      mbar_init(bar(BR::RING_EMPTY + s), 2);  // one commit from each MMA thread
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -330,13 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ring_last[s] >= 0) drain_wait(bar(BR::RING_FULL + s), (uint32_t)ring_last[s]);
         }
       }
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- tcgen05 issuer
+    } else if (warp == 1 || warp == 3) {
+      // ---------------------------------------------------------- tcgen05 issuers
+      // Two threads issue MMAs: warp 1 for query tile 0, warp 3 for tile 1.
+      // While one waits on a barrier the other keeps the tensor pipe's short
+      // queue fed. Both walk the same items and pages and follow the S
+      // buffer's owners in the same global order (S_0(t), S_1(t) per page), so
+      // each knows whose S_FREE to wait for; only data dependencies order the
+      // two threads' MMAs.
       if (lane == 0) {
-        // g: pages consumed; pv[w]: P.V MMAs issued for query tile w (= P_w
-        // buffers consumed); sc[w]: S MMAs issued for tile w; itw[w]: items
-        // done by tile w; s_last: tile whose S the buffer holds (-1: none).
-        uint32_t g = 0, it = 0, pv[2] = {0, 0}, sc[2] = {0, 0}, itw[2] = {0, 0};
+        const int mw = warp == 1 ? 0 : 1;  // the query tile this thread issues for
+        // g: pages walked; pv: P.V MMAs issued (P_mw buffers consumed);
+        // sc[w]: S MMAs issued so far for tile w (by either thread); itw:
+        // items done by tile mw; s_last: tile whose S the buffer holds.
+        uint32_t g = 0, it = 0, pv = 0, sc[2] = {0, 0}, itw = 0;
         int s_last = -1;
         bool ok = true;
         auto ring_wait = [&](uint32_t r, int code) -> bool {
@@ -351,14 +360,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
         auto lo_k = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | (1u << 16); };
         auto lo_mn = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | ((16384u >> 4) << 16); };
-        // S = Q_w K(t)^T into the S buffer, once the softmax warpgroup that
-        // owns the buffer's previous contents has loaded them.
-        auto issue_s = [&](int w, uint32_t t) -> bool {
+        // An S of tile w (ours or the other thread's) takes the buffer.
+        auto take_s = [&](int w) {
+          ++sc[w];
+          s_last = w;
+        };
+        // S = Q_mw K(t)^T into the S buffer, once the buffer's previous owner
+        // has loaded it.
+        auto issue_s = [&](uint32_t t) -> bool {
           if (s_last >= 0 &&
               !wait_bar(bar(B_S_FREE + s_last), (sc[s_last] - 1) & 1, ctl, 0x119 + s_last))
             return false;
           tc_fence_after();
-          const uint32_t qaddr = sbase + C::kQOff + w * C::kTileBytes;
+          const uint32_t qaddr = sbase + C::kQOff + mw * C::kTileBytes;
           const uint32_t kaddr = slot_addr(2 * t);
           if constexpr (D == 128) {
             mma_ss_k128<2, C::kPanelBytes / 16, 2, C::kPanelBytes / 16>(
@@ -371,32 +385,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                      kk > 0 ? 1u : 0u);
             }
           }
-          tc_commit(bar(B_S_FULL + w));
-          ++sc[w];
-          s_last = w;
+          tc_commit(bar(B_S_FULL + mw));
+          take_s(mw);
           return true;
         };
-        // O_w (+)= P_w V(t), P_w read from TMEM, once softmax w has written P_w
-        // (and, for an item's first P.V, once its epilogue has read O_w). The
-        // commit on P_FREE_w lets softmax w overwrite P_w (and touch O_w).
-        auto issue_pv = [&](int w, uint32_t t, bool accumulate, bool v_wait) -> bool {
-          if (!wait_bar(bar(B_P_FULL + w), pv[w] & 1, ctl, 0x112 + w)) return false;
-          if (!accumulate && itw[w] > 0 &&
-              !wait_bar(bar(B_O_EMPTY + w), (itw[w] - 1) & 1, ctl, 0x114 + w))
+        // O_mw (+)= P_mw V(t), once softmax mw has written P_mw (and, for an
+        // item's first P.V, once its epilogue has read O_mw) and V(t) is in.
+        // The commit on P_FREE_mw hands P_mw (and O_mw) back to the softmax.
+        auto issue_pv = [&](uint32_t t, bool accumulate) -> bool {
+          if (!wait_bar(bar(B_P_FULL + mw), pv & 1, ctl, 0x112 + mw)) return false;
+          if (!accumulate && itw > 0 &&
+              !wait_bar(bar(B_O_EMPTY + mw), (itw - 1) & 1, ctl, 0x114 + mw))
             return false;
-          if (v_wait && !ring_wait(2 * t + 1, 0x116)) return false;
+          if (!ring_wait(2 * t + 1, 0x116 + mw)) return false;
           tc_fence_after();
           const uint32_t vaddr = slot_addr(2 * t + 1);
-          mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * w, tmem + C::kColP + 64 * w,
+          mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * mw, tmem + C::kColP + 64 * mw,
                                  lo_mn(vaddr), kDescHi, C::kIdescO, accumulate ? 1u : 0u);
-          tc_commit(bar(B_P_FREE + w));
-          ++pv[w];
+          tc_commit(bar(B_P_FREE + mw));
+          ++pv;
           return true;
         };
-        // Pipe order per page t: S_0(t), PV_0(t-1), S_1(t), PV_1(t-1). A
-        // tile's P(t) is consumed after S of page t+1, so its softmax has the
-        // three other MMA groups in between; the S buffer is reloaded while
-        // the P.V behind it runs.
+        // A ring slot is released by one commit from each MMA thread; with a
+        // single query tile, thread 0 gives both.
+        auto release = [&](uint32_t r, int nq) {
+          tc_commit(bar(BR::RING_EMPTY + r % S));
+          if (nq == 1) tc_commit(bar(BR::RING_EMPTY + r % S));
+        };
+        // Pipe order per page t: S_0(t), PV_0(t-1) from thread 0 and S_1(t),
+        // PV_1(t-1) from thread 1. A tile's P(t) is consumed after S of page
+        // t+1, so its softmax has a whole page period; the S buffer is reloaded
+        // while the P.V behind it runs.
         for (uint32_t k = 0; ok; ++k) {
           int item;
           if (!next_item(k, 0x118, item)) { ok = false; break; }
@@ -405,35 +424,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Item w = decode_item(p, item);
           const int n = p.nodes[w.node].n_pages;
           const int nq = w.two ? 2 : 1;
-          if (!wait_bar(bar(B_Q_FULL), it & 1, ctl, 0x110)) { ok = false; break; }
+          const uint32_t qit = it++;
+          if (mw >= nq) {  // the item has no tile for this thread: follow the S chain only
+            for (int j = 0; j < n; ++j) take_s(0);
+            g += n;
+            continue;
+          }
+          if (!wait_bar(bar(B_Q_FULL), qit & 1, ctl, 0x110)) { ok = false; break; }
           for (int j = 0; j < n && ok; ++j, ++g) {
-            if (!ring_wait(2 * g, 0x111)) { ok = false; break; }
-            for (int q = 0; q < nq; ++q) {
-              if (!issue_s(q, g)) { ok = false; break; }
-              if (q == nq - 1) {
-                tc_commit(bar(BR::RING_EMPTY + (2 * g) % S));  // K(g) done
-                if (j == n - 1) tc_commit(bar(B_Q_EMPTY));
-              }
-              if (j > 0) {
-                if (!issue_pv(q, g - 1, j > 1, q == 0)) { ok = false; break; }
-                if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * (g - 1) + 1) % S));
-              }
+            if (mw == 1) take_s(0);  // thread 0's S_0(t) went first
+            // Thread 1's S follows S_0(t), whose S_FREE implies K(t) was in.
+            if (mw == 0 && !ring_wait(2 * g, 0x111)) { ok = false; break; }
+            if (!issue_s(g)) { ok = false; break; }
+            if (mw == nq - 1 && j == n - 1) tc_commit(bar(B_Q_EMPTY));  // the item's last S
+            release(2 * g, nq);  // K(t): this thread's S done
+            if (mw == 0 && nq == 2) take_s(1);  // thread 1's S_1(t) follows
+            if (j > 0) {
+              if (!issue_pv(g - 1, j > 1)) { ok = false; break; }
+              release(2 * (g - 1) + 1, nq);  // V(t-1): this thread's P.V done
             }
           }
           if (!ok) break;
-          // The item's last page: P.V of both tiles, then O is complete.
-          for (int q = 0; q < nq; ++q) {
-            if (!issue_pv(q, g - 1, n > 1, q == 0)) { ok = false; break; }
-            tc_commit(bar(B_O_FULL + q));
-            if (q == nq - 1) tc_commit(bar(BR::RING_EMPTY + (2 * (g - 1) + 1) % S));
-          }
-          if (!ok) break;
-          for (int q = 0; q < nq; ++q) ++itw[q];
-          ++it;
+          // The item's last page: this tile's P.V, then its O is complete.
+          if (!issue_pv(g - 1, n > 1)) { ok = false; break; }
+          tc_commit(bar(B_O_FULL + mw));
+          release(2 * (g - 1) + 1, nq);
+          ++itw;
         }
         // Wait (bounded) until every MMA issued by this thread has finished.
-        tc_commit(bar(B_DRAIN));
-        drain_wait(bar(B_DRAIN), 0);
+        tc_commit(bar(B_DRAIN + mw));
+        drain_wait(bar(B_DRAIN + mw), 0);
       }
     }
   } else {
