@@ -377,6 +377,16 @@ def run_gpu(args):
                 "frac": round(p_flops / (p_ms * 1e-3) / 1e12 / _measured_peaks()[0]["bf16_tflops"],
                               4)}
 
+    # ---- one whole transformer block of the round (Wan2.1-1.3B shapes, random
+    # weights): the round's QKV projection with the rotary embedding and the K/V
+    # append fused in (one launch for all nodes), the wave-round attention, the
+    # out-projection with the residual, the tanh-GELU MLP up and the MLP down
+    # with the residual. Events around every launch; a sleep kernel keeps the
+    # GPU busy while the host enqueues the first launches.
+    block = None
+    if spec.key == DEFAULT_WORKLOAD and not args.no_block:
+        block = block_round(wave, kv, wl, active, stream, args)
+
     # ---- end to end through the public API with host buffers. Every step copies
     # its Q and the round's K/V from pinned host memory and reads O back; the
     # copies of step i+1 run on their own streams while step i computes (device
@@ -471,6 +481,7 @@ def run_gpu(args):
                                  peaks["hbm_gbs"], 4)},
         "gpu_launches": K * 2,
         "projection": proj,
+        "block": block,
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and spec.key == DEFAULT_WORKLOAD:
@@ -480,6 +491,80 @@ def run_gpu(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def block_round(wave, kv, wl, active, stream, args):
+    """Time one transformer block of the round; per-kernel ms and TFLOP/s."""
+    import torch
+    C, F = wi.WAN21_DIM, wi.WAN21_MLP
+    n, T, H, d = len(active), wl.tokens, wl.heads, wl.head_dim
+    M = n * T
+    X = torch.cat([_bits_to_dev(wi.hidden_states(c, l, T, C)) for c, l in active])
+    Wq = _bits_to_dev(wi.qkv_weight(H, d, C))
+    Wo = _bits_to_dev(wi.block_weight("wo", C, H * d))
+    W1 = _bits_to_dev(wi.block_weight("w1", F, C))
+    W2 = _bits_to_dev(wi.block_weight("w2", C, F))
+    Q = torch.empty((M, H, d), dtype=torch.bfloat16, device="cuda")
+    A = torch.empty_like(Q)
+    Y = torch.empty((M, C), dtype=torch.bfloat16, device="cuda")
+    U = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    Z = torch.empty((M, C), dtype=torch.bfloat16, device="cuda")
+    names = ["qkv_rope_append", "attention", "out_proj", "mlp_up", "mlp_down"]
+    flops = [2 * M * 3 * H * d * C, None, 2 * M * C * H * d, 2 * M * F * C, 2 * M * C * F]
+
+    def one(ev=None):
+        steps = [
+            lambda: kv.qkv_append_round(active, X, Wq, Q, rope=wi.WAN21_GRID, stream=stream),
+            lambda: kv.round_attn(active, POLICY, Q, A, stream),
+            lambda: kv.linear(A.view(M, H * d), Wo, Y, R=X, stream=stream),
+            lambda: kv.linear(Y, W1, U, act=wave.ACT_GELU_TANH, stream=stream),
+            lambda: kv.linear(U, W2, Z, R=Y, stream=stream),
+        ]
+        for i, f in enumerate(steps):
+            if ev is not None:
+                ev[i].record(stream)
+            f()
+        if ev is not None:
+            ev[len(steps)].record(stream)
+        for nd in active:
+            kv.release(*nd)
+
+    one()  # the attention FLOPs come from the library's own key tables
+    kv.qkv_append_round(active, X, Wq, Q, rope=wi.WAN21_GRID, stream=stream)
+    table = kv.gather_table(active, POLICY)
+    for nd in active:
+        kv.release(*nd)
+    flops[1] = sum(4 * T * sum(v for _, v in rows) * H * d for rows in table)
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
+    torch.cuda._sleep(int(3e6))
+    for r in range(reps):
+        one(evs[r])
+    torch.cuda.synchronize()
+    kv.status(stream)
+    per = [[evs[r][i].elapsed_time(evs[r][i + 1]) for r in range(reps)] for i in range(5)]
+    total = [evs[r][0].elapsed_time(evs[r][5]) for r in range(reps)]
+    ms_round = statistics.median(total)
+    peak = _measured_peaks()[0]["bf16_tflops"]
+    kernels = {}
+    for i, name in enumerate(names):
+        ms = statistics.median(per[i])
+        tf = flops[i] / (ms * 1e-3) / 1e12
+        kernels[name] = {"ms": round(ms, 4), "flops": flops[i], "tflops": round(tf, 2),
+                         "frac": round(tf / peak, 4)}
+    upd = sum(1 for nd in active if nd[1] > 0)
+    return {"what": "one transformer block per round: QKV projection + rotary + K/V append "
+                    "(one launch for the round's nodes), wave attention, out-projection + "
+                    "residual, tanh-GELU MLP up, MLP down + residual; Wan2.1-1.3B shapes "
+                    f"(C {C}, MLP {F}, grid {wi.WAN21_GRID}), random weights",
+            "ms_per_round": round(ms_round, 4), "flops_per_round": sum(flops),
+            "tflops": round(sum(flops) / (ms_round * 1e-3) / 1e12, 2),
+            "chunk_updates_per_s": round(upd / (ms_round * 1e-3), 2),
+            "gemm_kernel": "gemm_wide_kernel", "kernels": kernels,
+            "peak_tflops": peak, "reps": reps}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -580,6 +665,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wave", "reference"], default="wave")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the whole-block round (projection, attention, MLP)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--clocks-csv", default=None,
                     help="keep the raw nvidia-smi samples here ({rank} is replaced); "

@@ -35,6 +35,14 @@ class Node(ctypes.Structure):
     _fields_ = [("chunk", ctypes.c_int32), ("level", ctypes.c_int32)]
 
 
+class Rope(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int32), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32),
+                ("base", ctypes.c_float)]
+
+
+ACT_NONE, ACT_GELU_TANH = 0, 1
+
+
 class KVConfig(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("tokens_per_chunk", ctypes.c_int32), ("num_levels", ctypes.c_int32),
@@ -55,6 +63,9 @@ _SIGS = {
                                       ctypes.c_void_p]),
     "wave_kv_release": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32]),
     "wave_kv_free_pages": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)]),
+    "wave_kv_entry_pages": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_int32)]),
     "wave_gather_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
                                          ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
                                          ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
@@ -71,6 +82,13 @@ _SIGS = {
     "wave_qkv_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "wave_qkv_append_round": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
+                                             ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                             ctypes.POINTER(Rope), ctypes.c_void_p,
+                                             ctypes.c_void_p]),
+    "wave_linear": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                                   ctypes.c_void_p, ctypes.c_void_p]),
     "wave_kv_append_batch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Node),
                                             ctypes.POINTER(ctypes.c_void_p),
                                             ctypes.POINTER(ctypes.c_void_p),
@@ -247,8 +265,45 @@ class KVCache:
                                         ctypes.c_void_p(Q.data_ptr()), _stream_handle(stream)))
         return Q
 
+    def qkv_append_round(self, nodes, X, W, Q, rope=None, stream=None):
+        """Project the round's nodes (X [n T][C], node i at rows i T) with W
+        [3 H d][C] into Q ([n T][H][d]) and each node's new K/V pages, Q and K
+        turned by ``rope`` = (frames, rows, cols[, base]) or not (None); one
+        kernel launch."""
+        r = None
+        if rope is not None:
+            f, rr, c = rope[:3]
+            base = rope[3] if len(rope) > 3 else 10000.0
+            r = ctypes.byref(Rope(f, rr, c, base))
+        _check(self.lib.wave_qkv_append_round(
+            self.h, _nodes(nodes), len(nodes), ctypes.c_void_p(X.data_ptr()), X.shape[1],
+            ctypes.c_void_p(W.data_ptr()), r, ctypes.c_void_p(Q.data_ptr()),
+            _stream_handle(stream)))
+        return Q
+
+    def linear(self, A, W, Y, R=None, act=ACT_NONE, stream=None):
+        """Y [M][N] = act(A W^T) (+ R) on the tensor cores; A [M][K], W [N][K]."""
+        M, K = A.shape[0], A.numel() // A.shape[0]
+        N = W.shape[0]
+        _check(self.lib.wave_linear(self.h, ctypes.c_void_p(A.data_ptr()), M, K,
+                                    ctypes.c_void_p(W.data_ptr()), N,
+                                    ctypes.c_void_p(R.data_ptr()) if R is not None else None,
+                                    int(act), ctypes.c_void_p(Y.data_ptr()),
+                                    _stream_handle(stream)))
+        return Y
+
     def release(self, chunk, level):
         _check(self.lib.wave_kv_release(self.h, chunk, level))
+
+    def entry_pages(self, chunk, level):
+        """Page ids of entry (chunk, level), in token order."""
+        n = ctypes.c_int32()
+        rc = self.lib.wave_kv_entry_pages(self.h, chunk, level, None, 0, ctypes.byref(n))
+        if rc not in (OK, ERR_CAPACITY):
+            _check(rc)
+        buf = (ctypes.c_int32 * max(1, n.value))()
+        _check(self.lib.wave_kv_entry_pages(self.h, chunk, level, buf, n.value, ctypes.byref(n)))
+        return list(buf[:n.value])
 
     def free_pages(self) -> int:
         n = ctypes.c_int32()

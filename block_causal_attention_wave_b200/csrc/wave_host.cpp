@@ -217,6 +217,19 @@ int wave_kv_release(wave_kv* kv, int32_t chunk, int32_t level) {
   return WAVE_OK;
 }
 
+int wave_kv_entry_pages(const wave_kv* kv, int32_t chunk, int32_t level, int32_t* pages,
+                        int32_t cap, int32_t* n) {
+  clear_error();
+  if (!kv || !n) return fail(WAVE_ERR_ARG, "NULL argument");
+  auto it = kv->entries.find(std::make_pair(chunk, level));
+  if (it == kv->entries.end())
+    return fail(WAVE_ERR_MISSING_KV, "(%d, %d) holds no K/V", chunk, level);
+  *n = (int32_t)it->second.pages.size();
+  if (*n > cap || !pages) return fail(WAVE_ERR_CAPACITY, "entry has %d pages, capacity %d", *n, cap);
+  std::memcpy(pages, it->second.pages.data(), *n * sizeof(int32_t));
+  return WAVE_OK;
+}
+
 int wave_kv_set_wait_limit(wave_kv* kv, uint64_t ns) {
   clear_error();
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");

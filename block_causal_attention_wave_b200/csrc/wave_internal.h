@@ -66,6 +66,13 @@ int check_current_device(const wave_kv* kv);
 uint64_t wait_limit_ns(const wave_kv* kv);
 // The driver's tensor-map encoder, looked up once (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+// The persistent 128 x 256 tcgen05 GEMM (wave_gemm.cu) in its QKV mode: the
+// projection of n nodes of T tokens each (rows i T .. of X) into Q and the
+// pages of their entries (already allocated), Q and K turned when rope is
+// non-null. Needs head_dim 128 and 3 * heads even (qkv_wide_supported).
+bool qkv_wide_supported(const wave_kv* kv);
+int qkv_wide_launch(wave_kv* kv, int32_t n, const wave_node* nodes, int32_t T, const void* X,
+                    int32_t dim, const void* W, const wave_rope* rope, void* Q, void* stream);
 // One kernel launch copying the K/V of n entries (already allocated) into
 // their pages.
 int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,

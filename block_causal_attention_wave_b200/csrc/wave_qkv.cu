@@ -10,10 +10,10 @@
 // producing side of the in-round K/V delivery of the Wave Forcing page ("Key
 // Findings"): the K/V reach the round's cache without a separate copy.
 //
-// How (two kernels). With d = 128 and 3 H even, qkv_append_wide_kernel (below)
-// takes tiles of 128 tokens x 256 features in persistent CTAs. Otherwise one
-// CTA per output tile of 128 tokens x one head's d features of Q, K or V --
-// for K and V exactly one page tile. 128 threads:
+// How. With d = 128 and 3 H even the projection runs on the persistent
+// 128 x 256 GEMM of wave_gemm.cu (its QKV mode). Otherwise (d = 64, or 3 H
+// odd) one CTA per output tile of 128 tokens x one head's d features of Q, K
+// or V -- for K and V exactly one page tile. 128 threads:
 //   warp 0 lane 0  TMA producer: 64-column slices of the X tile and the W tile
 //                  (both K-major, 128-byte swizzle) into a 3-stage ring;
 //   warp 1 lane 0  tcgen05 issuer: four M128 x Nd x K16 MMAs per slice into
@@ -73,8 +73,6 @@ struct QkvParams {
   int32_t heads;
   int32_t k_slices;     // C / 64
   int32_t n_mtiles;     // 128-token tiles = the entry's pages
-  int32_t n_pairs;      // 256-feature tiles (wide kernel): 3 H / 2
-  int32_t n_tiles;      // n_mtiles * n_pairs (wide kernel)
   int32_t pad;
   int32_t pages[WAVE_MAX_APPEND_PAGES];  // the entry's pages, one per 128 tokens
 };
@@ -194,194 +192,6 @@ __global__ void __launch_bounds__(kQkvThreads, 2) qkv_append_kernel(const __grid
   }
 }
 
-// ---------------------------------------------------------------------------
-// Wide variant (d = 128, 3 H even): output tiles of 128 tokens x 256 features
-// (two head slices of Q, K or V), one persistent CTA per SM walking its tiles
-// with two TMEM accumulators, so a tile's epilogue runs under the next tile's
-// MMAs. The 256-wide tile moves 96 KB through shared memory per 512 tensor
-// cycles (TMA in, MMAs out) instead of 64 KB per 256, which is what bounds the
-// 128-wide tile. 192 threads: warp 0 TMA, warp 1 MMA (and TMEM), warps 2..5
-// epilogue (warp w reads TMEM lanes 32 (w % 4) ..).
-constexpr int kWideThreads = 192;
-constexpr int kWideStages = 4;
-
-struct WideCfg {
-  static constexpr int kATile = 128 * 128;  // 128 token rows x 64 bf16
-  static constexpr int kBTile = 256 * 128;  // 256 weight rows x 64 bf16
-  static constexpr int kStage = kATile + kBTile;
-  static constexpr int kBarOff = kWideStages * kStage;
-  // FULL[s], EMPTY[s], ACC_FULL[2], ACC_EMPTY[2], DRAIN
-  static constexpr int kFull = 0, kEmpty = kWideStages, kAccFull = 2 * kWideStages,
-                       kAccEmpty = kAccFull + 2, kDrain = kAccEmpty + 2, kBars = kDrain + 1;
-  static constexpr int kSmemBytes = kBarOff + 128 + 1024;
-  static_assert(kBars * 8 + 8 <= 128, "barrier area");
-  static constexpr uint32_t kIdesc =
-      (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
-};
-
-__global__ void __launch_bounds__(kWideThreads, 1)
-    qkv_append_wide_kernel(const __grid_constant__ QkvParams p) {
-  using C = WideCfg;
-  constexpr int S = kWideStages;
-  constexpr int D = 128;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const uint32_t sb = smem_addr(smem);
-  auto bar = [&](int i) -> uint32_t { return sb + C::kBarOff + 8u * i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * C::kBars + 4);
-  const Ctl ctl{abort_flag, p.status, p.wait_ns};
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = p.k_slices, n_tiles = p.n_tiles, n_m = p.n_mtiles;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(bar(C::kFull + s), 1);
-      mbar_init(bar(C::kEmpty + s), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(bar(C::kAccFull + a), 1);
-      mbar_init(bar(C::kAccEmpty + a), 128);
-    }
-    mbar_init(bar(C::kDrain), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    prefetch_tmap(&p.tm_x);
-    prefetch_tmap(&p.tm_w);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // Producer: slices of every tile of this CTA through one ring.
-      uint32_t g = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int pr = t / n_m, m = t - pr * n_m;
-        for (int k = 0; k < nk; ++k, ++g) {
-          const uint32_t s = g % S;
-          if (g >= (uint32_t)S &&
-              !wait_bar(bar(C::kEmpty + s), ((g / S) - 1) & 1, ctl, 0x211)) {
-            ok = false;
-            break;
-          }
-          const uint32_t a = sb + s * C::kStage;
-          mbar_arrive_expect_tx(bar(C::kFull + s), C::kStage);
-          tma_load_2d(a, &p.tm_x, k * 64, m * 128, bar(C::kFull + s));
-          tma_load_2d(a + C::kATile, &p.tm_w, k * 64, pr * 256, bar(C::kFull + s));
-        }
-      }
-      for (uint32_t k = g > (uint32_t)S ? g - S : 0; k < g; ++k)
-        drain_wait(bar(C::kFull + k % S), (k / S) & 1);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // MMA issuer: tile i of this CTA accumulates in TMEM columns 256 (i % 2).
-      uint32_t g = 0, i = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
-        const uint32_t acc = i & 1;
-        if (i >= 2 && !wait_bar(bar(C::kAccEmpty + acc), ((i >> 1) - 1) & 1, ctl, 0x212)) break;
-        tc_fence_after();
-        for (int k = 0; k < nk; ++k, ++g) {
-          const uint32_t s = g % S;
-          if (!wait_bar(bar(C::kFull + s), (g / S) & 1, ctl, 0x213)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a = sb + s * C::kStage;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + 256 * acc, desc_k(a + kk * 32), desc_k(a + C::kATile + kk * 32),
-                   C::kIdesc, (k | kk) != 0 ? 1u : 0u);
-          tc_commit(bar(C::kEmpty + s));
-        }
-        if (ok) tc_commit(bar(C::kAccFull + acc));
-      }
-      // Every MMA issued above completes before TMEM is released.
-      tc_commit(bar(C::kDrain));
-      drain_wait(bar(C::kDrain), 0);
-    }
-  } else {
-    // Epilogue: thread r of warps 2..5 owns token row r of each tile.
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint32_t i = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
-      const uint32_t acc = i & 1;
-      const bool ok = __all_sync(0xffffffffu, wait_bar(bar(C::kAccFull + acc), (i >> 1) & 1, ctl, 0x214));
-      if (!ok) break;
-      tc_fence_after();
-      const int pr = t / n_m, m = t - pr * n_m;
-      const int token = m * 128 + row;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int n = 2 * pr + h;
-        const int which = n / p.heads, head = n - which * p.heads;
-        uint4* dst;
-        bool store;
-        if (which == 0) {
-          dst = reinterpret_cast<uint4*>(p.q + ((int64_t)token * p.heads + head) * D);
-          store = token < p.ntokens;
-        } else {
-          dst = reinterpret_cast<uint4*>(p.data + (int64_t)p.pages[m] * p.page_bytes +
-                                         ((((int64_t)(which - 1) * p.heads + head) * 128 + row) * D) * 2);
-          store = true;  // rows past the tokens hold zeros: the page tail
-        }
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + 256 * acc + 128 * h + 32 * c, v);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          if (store) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[c * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::kAccEmpty + acc));
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-int launch_qkv_wide(const QkvParams& prm, int grid, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(qkv_append_wide_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, WideCfg::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess)
-    return fail(WAVE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  qkv_append_wide_kernel<<<grid, kWideThreads, WideCfg::kSmemBytes, stream>>>(prm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess)
-    return fail(WAVE_ERR_CUDA, "qkv_append_wide_kernel launch: %s", cudaGetErrorString(e));
-  return WAVE_OK;
-}
-
 template <int D>
 int launch_qkv(const QkvParams& prm, dim3 grid, cudaStream_t stream) {
   static std::once_flag once;
@@ -398,9 +208,12 @@ int launch_qkv(const QkvParams& prm, dim3 grid, cudaStream_t stream) {
   return WAVE_OK;
 }
 
-int qkv_append_impl(wave_kv* kv, const wave_entry& ent, const void* X, int32_t dim,
-                    const void* W, void* Q, void* stream) {
+int qkv_append_impl(wave_kv* kv, wave_node node, const wave_entry& ent, const void* X,
+                    int32_t dim, const void* W, void* Q, void* stream) {
   const int H = kv->cfg.heads, D = kv->cfg.head_dim;
+  // d = 128 with 3 H even: the persistent 128 x 256 GEMM of wave_gemm.cu.
+  if (qkv_wide_supported(kv))
+    return qkv_wide_launch(kv, 1, &node, ent.ntokens, X, dim, W, nullptr, Q, stream);
   static thread_local QkvParams prm;
   std::memset(&prm, 0, offsetof(QkvParams, pages));
   auto encode = tensor_map_encoder();
@@ -416,11 +229,10 @@ int qkv_append_impl(wave_kv* kv, const wave_entry& ent, const void* X, int32_t d
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled(X) failed: %d", (int)r);
   }
-  const bool wide = D == 128 && (3 * H) % 2 == 0;
   {
     cuuint64_t dims[2] = {(cuuint64_t)dim, (cuuint64_t)3 * H * D};
     cuuint64_t strides[1] = {(cuuint64_t)dim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)(wide ? 256 : D)};
+    cuuint32_t box[2] = {64, (cuuint32_t)D};
     CUresult r = encode(&prm.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -439,11 +251,6 @@ int qkv_append_impl(wave_kv* kv, const wave_entry& ent, const void* X, int32_t d
   std::memcpy(prm.pages, ent.pages.data(), n_pages * sizeof(int32_t));
   prm.n_mtiles = n_pages;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (wide) {
-    prm.n_pairs = 3 * H / 2;
-    prm.n_tiles = n_pages * prm.n_pairs;
-    return launch_qkv_wide(prm, std::min(prm.n_tiles, kv->num_sms), s);
-  }
   dim3 grid((unsigned)n_pages, (unsigned)(3 * H));
   return D == 128 ? launch_qkv<128>(prm, grid, s) : launch_qkv<64>(prm, grid, s);
 }
@@ -472,7 +279,7 @@ extern "C" int wave_qkv_append(wave_kv* kv, int32_t chunk, int32_t level, const 
   int rc = wave_kv_alloc(kv, chunk, level, ntokens);
   if (rc) return rc;
   const wave_entry& e = kv->entries.at(std::make_pair(chunk, level));
-  rc = qkv_append_impl(kv, e, X, dim, W, Q, stream);
+  rc = qkv_append_impl(kv, wave_node{chunk, level}, e, X, dim, W, Q, stream);
   if (rc) {
     std::string keep = wave_last_error_detail();
     wave_kv_release(kv, chunk, level);

@@ -156,12 +156,77 @@ int wave_kv_append_batch(wave_kv* kv, int32_t n_entries, const wave_node* entrie
 int wave_qkv_append(wave_kv* kv, int32_t chunk, int32_t level, const void* X, int32_t ntokens,
                     int32_t dim, const void* W, void* Q, void* stream);
 
+/* Rotary position embedding of a chunk's tokens over three axes of the video
+ * latent (frame, row, column): token t of chunk c sits at frame
+ * c * frames + t / (rows * cols), row (t / cols) % rows, column t % cols. Of
+ * the d/2 rotation pairs of a head (elements 2p, 2p+1) the first
+ * d/2 - 2 (d/6) turn with the frame, the next d/6 with the row and the last
+ * d/6 with the column (integer division); pair i of a group of n pairs turns
+ * by position * base^(-i/n) radians: (a, b) -> (a cos - b sin, a sin + b cos).
+ * The pages give no positional scheme; this is the reading of a rotary
+ * embedding on the latent grid of the chunks they describe ([DS] Appendix
+ * Table 4: 3 latent frames of 832x480 per chunk). */
+typedef struct {
+  int32_t frames; /* F: latent frames per chunk                        */
+  int32_t rows;   /* R: token rows per frame                           */
+  int32_t cols;   /* W: token columns per frame; F * R * W = T          */
+  float base;     /* frequency base, > 1 (10000 in common use)         */
+} wave_rope;
+
+/* The QKV projection of ALL n_nodes nodes of a round in ONE kernel launch,
+ * with the rotary embedding of Q and K and the K/V append fused into its
+ * epilogue: for node i = nodes[i], [Q | K | V] = X_i W^T (fp32 accumulation),
+ * Q and K turned by `rope` (NULL: no rotation), Q rounded to bf16 into the
+ * caller's buffer, K and V rounded to bf16 straight into the node's new cache
+ * entry (the pages and bytes wave_kv_alloc + wave_kv_append would give,
+ * zero page tail). This is the producing side of the in-round K/V delivery of
+ * [WF] ("Key Findings") for one transformer block of a round.
+ * X: device bf16 [n_nodes * T][dim], node i's hidden states at rows i*T;
+ * W: device bf16 [3*H*d][dim] (output feature (s*H + h)*d + j is Q (s = 0), K
+ * (s = 1) or V (s = 2) of head h, component j); Q: device bf16
+ * [n_nodes * T][H][d], written (node i at rows i*T, the layout
+ * wave_round_attn reads). All caller-owned, contiguous, 16-byte aligned; dim a
+ * multiple of 64; T = tokens_per_chunk. Needs head_dim 128 and 3*H even
+ * (UNSUPPORTED otherwise). Pages are taken in node order, lowest free first.
+ * Errors: ARG (pointers, dim, rope grid not covering T), EXISTS, NO_PAGES,
+ * CAPACITY (more than WAVE_MAX_APPEND_PAGES pages or WAVE_MAX_NODES nodes),
+ * UNSUPPORTED, CUDA; on any error no pages stay taken. A device-side timeout
+ * is reported by wave_kv_status. */
+int wave_qkv_append_round(wave_kv* kv, const wave_node* nodes, int32_t n_nodes, const void* X,
+                          int32_t dim, const void* W, const wave_rope* rope, void* Q,
+                          void* stream);
+
+#define WAVE_ACT_NONE      0
+#define WAVE_ACT_GELU_TANH 1 /* 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) */
+
+/* A dense layer of the round's transformer block on the tensor cores:
+ * Y = act(A W^T) (+ R), fp32 accumulation, bf16 result -- the out-projection
+ * (Y = X + attention W_o^T) and the two MLP products (U = GELU(Y W_1^T),
+ * Z = Y + U W_2^T) of one concurrent forward round ([WF] "Key Findings"; the
+ * pages give no formula for the block, these are the plain readings).
+ * A: device bf16 [M][K]; W: device bf16 [N][K] (a linear layer's [out][in]
+ * weight); R: device bf16 [M][N] residual or NULL (added after act); Y:
+ * device bf16 [M][N], written (may be R itself). All caller-owned,
+ * contiguous, 16-byte aligned. K a multiple of 64, N a multiple of 256,
+ * K, N <= 65536. `kv` names the device handle whose status word records a
+ * timeout (wave_kv_status) and whose device must be current; the pool itself
+ * is not touched. Errors: ARG, CUDA. */
+int wave_linear(wave_kv* kv, const void* A, int32_t M, int32_t K, const void* W, int32_t N,
+                const void* R, int32_t act, void* Y, void* stream);
+
 /* Return the pages of (chunk, level) to the free set. Host only; the caller
  * must not release an entry that queued device work still reads (all library
  * kernels read the pool in stream order, so releasing after enqueueing the
  * last reader on the same stream is safe when the next writer uses that
  * stream too). Errors: MISSING_KV. */
 int wave_kv_release(wave_kv* kv, int32_t chunk, int32_t level);
+
+/* Page ids of entry (chunk, level) in token order (page j holds tokens
+ * 128 j .. 128 j + 127; rows past the entry's tokens are zero once written).
+ * `cap` = capacity of pages; *n = the entry's page count. Host only.
+ * Errors: ARG, MISSING_KV, CAPACITY (cap too small; *n = pages needed). */
+int wave_kv_entry_pages(const wave_kv* kv, int32_t chunk, int32_t level, int32_t* pages,
+                        int32_t cap, int32_t* n);
 
 /* Number of free pages. */
 int wave_kv_free_pages(const wave_kv* kv, int32_t* n);

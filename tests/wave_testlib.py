@@ -101,3 +101,22 @@ def assert_close(got, want, what="", scale_with_output=False):
     bound = MAX_ABS * max(1.0, float(np.abs(want).max())) if scale_with_output else MAX_ABS
     assert max_abs <= bound and rel <= REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
     return max_abs, rel
+
+
+def read_entry(kv, pool, entry, tokens):
+    """K and V of one cache entry read back from the pool: ([T][H][d] float64
+    each, bf16 values) and whether the rows past the tokens are all zero."""
+    page_bytes, off, _ = kv.layout()
+    H, d = kv.heads, kv.head_dim
+    host = pool.cpu().numpy()
+    pages = kv.entry_pages(*entry)
+    out, tail_zero = [], True
+    for kvi in range(2):
+        rows = np.zeros((len(pages) * 128, H, d), dtype=np.uint16)
+        for pi, page in enumerate(pages):
+            base = off + page * page_bytes + kvi * H * 128 * d * 2
+            blk = host[base:base + H * 128 * d * 2].view(np.uint16)
+            rows[pi * 128:(pi + 1) * 128] = blk.reshape(H, 128, d).transpose(1, 0, 2)
+        tail_zero = tail_zero and not rows[tokens:].any()
+        out.append(wi.bf16_bits_to_f64(rows[:tokens]))
+    return out[0], out[1], tail_zero

@@ -67,6 +67,22 @@ def qkv_weight(heads: int, head_dim: int, dim: int) -> np.ndarray:
     return normal_bf16(PROJ_SEED_BASE - 1, (3 * heads * head_dim, dim), 1.0 / math.sqrt(dim))
 
 
+_BLOCK_WEIGHTS = {"wo": 2, "w1": 3, "w2": 4}
+
+
+def block_weight(name: str, out_dim: int, in_dim: int) -> np.ndarray:
+    """``[out_dim][in_dim]`` bf16 bits of N(0, 1) / sqrt(in_dim): a random weight
+    of the block's out-projection ("wo") or MLP ("w1", "w2"), [out][in] layout."""
+    return normal_bf16(PROJ_SEED_BASE - _BLOCK_WEIGHTS[name], (out_dim, in_dim),
+                       1.0 / math.sqrt(in_dim))
+
+
+# Wan2.1-1.3B block: hidden size 1536 (12 heads x 128), MLP width 8960; a chunk
+# is 3 latent frames of 30 x 52 patch tokens.
+WAN21_DIM, WAN21_MLP = 1536, 8960
+WAN21_GRID = (3, 30, 52)
+
+
 def node_tensor(kind: str, chunk: int, level: int, tokens: int, heads: int,
                 head_dim: int, scale: float = 1.0) -> np.ndarray:
     """Token-major ``[tokens][heads][head_dim]`` bf16 bits for one (chunk, level)."""
