@@ -25,6 +25,9 @@ What it computes, each part written as the plain definition from the pages:
                                (frame, row, column), out-projection and
                                tanh-GELU MLP with residuals, bf16 storage
                                between kernels (readings stated there).
+* ``parallel``              -- Wave Parallelism host logic: node placement on
+                               ranks, one-way K/V pushes per round, and each
+                               rank's page tables.
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
 against something other than itself (brute-force dense masks, closed forms,
@@ -32,4 +35,4 @@ torch's CPU attention, exhaustive search). Absolute attention values printed by
 the pages: none exist, so that part is "parity unpinned" against the pages and
 pinned only by the mathematics.
 """
-from . import policy, schedule, cache, attention, projection, block  # noqa: F401
+from . import policy, schedule, cache, attention, projection, block, parallel  # noqa: F401
