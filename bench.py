@@ -387,6 +387,13 @@ def run_gpu(args):
     if spec.key == DEFAULT_WORKLOAD and not args.no_block:
         block = block_round(wave, kv, wl, active, stream, args)
 
+    # ---- split-KV attention (key lists cut into ranges, partials combined):
+    # the same round with the automatic range count, and a round of a single
+    # update node (few work items: the case the ranges are for).
+    split = None
+    if spec.key == "wan-streamer":
+        split = split_rounds(wave, kv, wl, active, dq, do, stream, flops)
+
     # ---- end to end through the public API with host buffers. Every step copies
     # its Q and the round's K/V from pinned host memory and reads O back; the
     # copies of step i+1 run on their own streams while step i computes (device
@@ -482,6 +489,7 @@ def run_gpu(args):
         "gpu_launches": K * 2,
         "projection": proj,
         "block": block,
+        "split_kv": split,
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and spec.key == DEFAULT_WORKLOAD:
@@ -491,6 +499,57 @@ def run_gpu(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def split_rounds(wave, kv, wl, active, dq, do, stream, flops):
+    """Time wave_round_attn_split (automatic ranges) against wave_round_attn
+    on the timed round and on its last update node alone."""
+    import torch
+    out = {}
+    T = wl.tokens
+    upd = [n for n in active if n[1] > 0][-1:]
+    kv.append_batch(active, *_round_kv(wl, active), stream)
+    one_flops = None
+    for name, nodes in (("round", active), ("one_node", upd)):
+        idx = [active.index(n) for n in nodes]
+        q = torch.cat([dq[i * T:(i + 1) * T] for i in idx])
+        o = torch.empty_like(q)
+        nbytes, used = kv.split_workspace(nodes, POLICY, 0)
+        wsb = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+        if name == "one_node":
+            table = kv.gather_table(nodes, POLICY)
+            f = sum(4 * T * sum(v for _, v in rows) * wl.heads * wl.head_dim for rows in table)
+        else:
+            f = flops
+        res = {"nodes": [list(n) for n in nodes], "flops": f, "splits": used}
+        for key, call in (("plain", lambda: kv.round_attn(nodes, POLICY, q, o, stream)),
+                          ("split", lambda: kv.round_attn_split(nodes, POLICY, q, o, wsb, 0,
+                                                                stream))):
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            torch.cuda._sleep(int(2e6))
+            ev[0].record(stream)
+            for _ in range(10):
+                call()
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            ms = ev[0].elapsed_time(ev[1]) / 10
+            res[key] = {"ms": round(ms, 4), "tflops": round(f / (ms * 1e-3) / 1e12, 2)}
+        out[name] = res
+    kv.status(stream)
+    for n in active:
+        kv.release(*n)
+    return out
+
+
+def _round_kv(wl, active):
+    ks = [_bits_to_dev(wi.node_tensor("k", c, l, wl.tokens, wl.heads, wl.head_dim, wl.scale))
+          for c, l in active]
+    vs = [_bits_to_dev(wi.node_tensor("v", c, l, wl.tokens, wl.heads, wl.head_dim, wl.scale))
+          for c, l in active]
+    return ks, vs
 
 
 def block_round(wave, kv, wl, active, stream, args):

@@ -43,6 +43,11 @@ class Rope(ctypes.Structure):
 ACT_NONE, ACT_GELU_TANH = 0, 1
 
 
+class Transfer(ctypes.Structure):
+    _fields_ = [("chunk", ctypes.c_int32), ("level", ctypes.c_int32), ("src", ctypes.c_int32),
+                ("dst", ctypes.c_int32)]
+
+
 class KVConfig(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("tokens_per_chunk", ctypes.c_int32), ("num_levels", ctypes.c_int32),
@@ -77,6 +82,15 @@ _SIGS = {
                                                       ctypes.c_int32, ctypes.c_int32,
                                                       ctypes.c_void_p, ctypes.c_void_p,
                                                       ctypes.c_void_p]),
+    "wave_round_attn_split": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node), ctypes.c_int32,
+                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64,
+                                             ctypes.c_void_p]),
+    "wave_round_attn_split_workspace": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Node),
+                                                       ctypes.c_int32, ctypes.c_int32,
+                                                       ctypes.c_int32,
+                                                       ctypes.POINTER(ctypes.c_uint64),
+                                                       ctypes.POINTER(ctypes.c_int32)]),
     "wave_kv_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "wave_kv_set_wait_limit": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64]),
     "wave_qkv_append": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
@@ -104,6 +118,14 @@ _SIGS = {
     "wave_schedule_last_read": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, ctypes.POINTER(Node),
                                                ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
+    "wave_wp_transfers": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.POINTER(Transfer), ctypes.c_int32,
+                                         ctypes.POINTER(ctypes.c_int32)]),
+    "wave_wp_rank_last_read": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.POINTER(Node), ctypes.c_int32,
+                                              ctypes.POINTER(ctypes.c_int32)]),
     "wave_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "wave_last_error_detail": (ctypes.c_char_p, []),
 }
@@ -186,6 +208,30 @@ def last_read_rounds(B: int, K: int, policy="progressive", window: int = 0, node
     out = (ctypes.c_int32 * max(1, len(nodes)))()
     _check(lib.wave_schedule_last_read(B, K, _policy(policy), window, arr, len(nodes), out))
     return {tuple(n): out[i] for i, n in enumerate(nodes)}
+
+
+def wp_transfers(B: int, K: int, policy, window: int, n_ranks: int, round_index: int):
+    """Wave Parallelism pushes of one round: [((chunk, level), src, dst), ...]."""
+    lib = load()
+    n = ctypes.c_int32(0)
+    rc = lib.wave_wp_transfers(B, K, _policy(policy), window, n_ranks, round_index, None, 0,
+                               ctypes.byref(n))
+    if rc not in (OK, ERR_CAPACITY):
+        _check(rc)
+    buf = (Transfer * max(1, n.value))()
+    _check(lib.wave_wp_transfers(B, K, _policy(policy), window, n_ranks, round_index, buf,
+                                 n.value, ctypes.byref(n)))
+    return [((t.chunk, t.level), t.src, t.dst) for t in buf[:n.value]]
+
+
+def wp_rank_last_read(B: int, K: int, policy, window: int, n_ranks: int, rank: int, entries):
+    """Dict entry -> last round in which a node of ``rank`` reads it."""
+    lib = load()
+    arr = _nodes(entries)
+    out = (ctypes.c_int32 * max(1, len(entries)))()
+    _check(lib.wave_wp_rank_last_read(B, K, _policy(policy), window, n_ranks, rank, arr,
+                                      len(entries), out))
+    return {tuple(e): out[i] for i, e in enumerate(entries)}
 
 
 class KVCache:
@@ -331,6 +377,26 @@ class KVCache:
         _check(self.lib.wave_round_attn(self.h, nodes, len(active), _policy(policy),
                                         ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(O.data_ptr()),
                                         _stream_handle(stream)))
+        return O
+
+    def split_workspace(self, active, policy, splits=0):
+        """(bytes, ranges per item) that round_attn_split needs."""
+        b, ns = ctypes.c_uint64(0), ctypes.c_int32(0)
+        _check(self.lib.wave_round_attn_split_workspace(self.h, _nodes(active), len(active),
+                                                        _policy(policy), int(splits),
+                                                        ctypes.byref(b), ctypes.byref(ns)))
+        return b.value, ns.value
+
+    def round_attn_split(self, active, policy, Q, O, workspace=None, splits=0, stream=None):
+        """round_attn with key lists cut into ranges (0 = automatic count);
+        ``workspace`` is a CUDA tensor of at least split_workspace() bytes."""
+        ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+        nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        _check(self.lib.wave_round_attn_split(self.h, _nodes(active), len(active),
+                                              _policy(policy), int(splits),
+                                              ctypes.c_void_p(Q.data_ptr()),
+                                              ctypes.c_void_p(O.data_ptr()), ptr, nbytes,
+                                              _stream_handle(stream)))
         return O
 
     def round_attn_static_scratch(self, active, policy, Q, O, stream=None):

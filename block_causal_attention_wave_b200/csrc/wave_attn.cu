@@ -82,6 +82,7 @@ struct AttnNode {
   int32_t item0;     // first work item
   int32_t n_pairs;   // ceil(n_qtiles / 2): pairs of 128-row query tiles
   int32_t n_qtiles;  // ceil(T / 128)
+  int32_t n_splits;  // key ranges per (head, pair); > 1: partial results
 };
 
 struct AttnParams {
@@ -91,6 +92,8 @@ struct AttnParams {
   int32_t* status;    // device status word (pool header)
   int32_t* counter;   // work-queue counter, zero at launch (pool header)
   int64_t* clock_out; // CTA 0's SM cycles and nanoseconds (pool header)
+  float* part_o;      // split key ranges: unnormalised O per (item, tile, row), fp32
+  float* part_ml;     // ... and the row's (running max, sum), fp32
   uint64_t wait_ns;   // bound on one barrier wait
   float scale_log2;   // log2(e) / sqrt(d)
   int32_t heads;
@@ -154,27 +157,33 @@ enum : int {
   B_RING_FULL = B_ITEM_EMPTY + 2,  // kSlots each from here
 };
 constexpr int kItemSlots = 2;
+constexpr int kItemWords = 8;  // an Item as published in the shared-memory queue
 
 template <int D>
 struct Bars {
   static constexpr int kS = Cfg<D>::kSlots;
   static constexpr int RING_FULL = B_RING_FULL, RING_EMPTY = RING_FULL + kS,
                        COUNT = RING_EMPTY + kS;
-  static_assert(COUNT * 8 + 16 + 4 * kItemSlots <= 448, "barrier area");  // 448..463: clock
+  static_assert(COUNT * 8 + 16 + 4 * kItemWords * kItemSlots <= 448, "barrier area");  // 448..: clock
 };
 
+// A work item: (node, head, pair of 128-row query tiles, key range). The
+// producer decodes it once and publishes these fields to the other roles.
 struct Item {
-  int node, head, pair;
-  bool two;  // the pair's second query tile holds rows of the node
+  int id, node, head, pair, two, page_begin, n_pages, split;
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   int n = 0;
   while (n + 1 < p.n_nodes && item >= p.nodes[n + 1].item0) ++n;
-  const int j = item - p.nodes[n].item0;
-  const int np = p.nodes[n].n_pairs;
-  const int pair = j % np;
-  return Item{n, j / np, pair, 2 * pair + 1 < p.nodes[n].n_qtiles};
+  const AttnNode& nd = p.nodes[n];
+  const int j = item - nd.item0;
+  const int ns = nd.n_splits;
+  const int split = j % ns, hp = j / ns;  // key ranges of one (head, pair) are adjacent
+  const int pair = hp % nd.n_pairs;
+  const int base = nd.n_pages / ns, extra = nd.n_pages % ns;
+  return Item{item, n, hp / nd.n_pairs, pair, 2 * pair + 1 < nd.n_qtiles ? 1 : 0,
+              split * base + min(split, extra), base + (split < extra ? 1 : 0), split};
 }
 
 // 2^x for a pair of x <= 8 on the FMA pipe: x = j + f, j = round(x),
@@ -267,10 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // producer claims the next one (the CTA's first is blockIdx.x, later ones
   // come from a global counter) and publishes it to the other roles through a
   // two-slot queue in shared memory. An id >= n_items tells every role to stop.
-  auto next_item = [&](uint32_t k, int code, int& item) -> bool {  // consumer side
+  auto next_item = [&](uint32_t k, int code, Item& w) -> bool {  // consumer side
     if (!wait_bar(bar(B_ITEM_FULL + (k % kItemSlots)), (k / kItemSlots) & 1, ctl, code))
       return false;
-    item = item_q[k % kItemSlots];
+    const volatile int* q = item_q + kItemWords * (k % kItemSlots);
+    w = Item{q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]};
     return true;
   };
 
@@ -293,10 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.counter, 1);
-          item_q[slot] = item;
+          Item w{item, 0, 0, 0, 0, 0, 0, 0};
+          if (item < p.n_items) w = decode_item(p, item);
+          volatile int* q = item_q + kItemWords * slot;
+          q[0] = w.id; q[1] = w.node; q[2] = w.head; q[3] = w.pair;
+          q[4] = w.two; q[5] = w.page_begin; q[6] = w.n_pages; q[7] = w.split;
           mbar_arrive(bar(B_ITEM_FULL + slot));
           if (item >= p.n_items) break;
-          const Item w = decode_item(p, item);
           const AttnNode& nd = p.nodes[w.node];
           if (it > 0 && !wait_bar(bar(B_Q_EMPTY), (it - 1) & 1, ctl, 0x101)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_Q_FULL), (w.two ? 2 : 1) * C::kTileBytes);
@@ -306,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           pn * 64, w.head, nd.q_row0 + (2 * w.pair + q) * 128, bar(B_Q_FULL));
           q_last = it & 1;
           ++it;
-          for (int t = 0; ok && t < nd.n_pages; ++t) {
-            const uint32_t page = p.pages[nd.page0 + t] & kPageMask;
+          for (int t = 0; ok && t < w.n_pages; ++t) {
+            const uint32_t page = p.pages[nd.page0 + w.page_begin + t] & kPageMask;
             const int32_t yk = (int32_t)(((int64_t)page * 2 * H + w.head) * 128);
             for (int kv = 0; kv < 2; ++kv, ++r) {
               const int s = r % S;
@@ -417,12 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // t+1, so its softmax has a whole page period; the S buffer is reloaded
         // while the P.V behind it runs.
         for (uint32_t k = 0; ok; ++k) {
-          int item;
-          if (!next_item(k, 0x118, item)) { ok = false; break; }
+          Item w;
+          if (!next_item(k, 0x118, w)) { ok = false; break; }
           mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
-          if (item >= p.n_items) break;
-          const Item w = decode_item(p, item);
-          const int n = p.nodes[w.node].n_pages;
+          if (w.id >= p.n_items) break;
+          const int n = w.n_pages;
           const int nq = w.two ? 2 : 1;
           const uint32_t qit = it++;
           if (mw >= nq) {  // the item has no tile for this thread: follow the S chain only
@@ -471,21 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P_FREE_w), it: items finished by this warpgroup.
     uint32_t g = 0, pw = 0, it = 0;
     for (uint32_t k = 0;; ++k) {
-      int item;
-      bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, item));
+      Item w;
+      bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, w));
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
-      if (item >= p.n_items) break;
-      const Item w = decode_item(p, item);
+      if (w.id >= p.n_items) break;
       if (wq == 1 && !w.two) continue;  // the pair's second tile lies past the node
       const AttnNode& nd = p.nodes[w.node];
       float m_run = -INFINITY, l_run = 0.f;
-      for (int t = 0; t < nd.n_pages; ++t, ++g) {
+      for (int t = 0; t < w.n_pages; ++t, ++g) {
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
         tc_fence_after();
-        const int valid = (int)(p.pages[nd.page0 + t] >> 25) + 1;
+        const int valid = (int)(p.pages[nd.page0 + w.page_begin + t] >> 25) + 1;
         // The whole S row in one TMEM round trip; then the S buffer goes back
         // to the MMA thread for the other tile's (or the next page's) S.
         float sv[128];
@@ -596,6 +607,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, wait_bar(bar(B_O_FULL + wq), it & 1, ctl, 0x122 + wq));
       if (!ok) break;
       tc_fence_after();
+      if (nd.n_splits > 1) {
+        // One key range of several: the unnormalised O row and its (running
+        // max, sum), both relative to the same max, for the combine kernel.
+        const int64_t slot = ((int64_t)w.id * 2 + wq) * 128 + row;
+        float4* po = reinterpret_cast<float4*>(p.part_o + slot * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            po[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                        __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+        reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_run, l_run);
+        tc_fence_before();
+        mbar_arrive(bar(B_O_EMPTY + wq));
+        ++it;
+        continue;
+      }
       const float inv = 1.f / l_run;
       const int q_local = (2 * w.pair + wq) * 128 + row;
       const bool store = q_local < p.q_rows;
@@ -635,6 +667,82 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Combine of split key ranges: for each query row of a node whose key list
+// was cut into S ranges, O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
+// with M = max_s m_s (the m_s are the ranges' running maxima in the log2
+// domain; each O_s and l_s is relative to its own m_s). One warp per query
+// row (eight rows per CTA, kCombineRowsPerCta), so thousands of rows' loads
+// are in flight at once; lane s holds range s's (m, l), and lanes split the d
+// values of O.
+struct CombineParams {
+  const float* part_o;
+  const float* part_ml;
+  uint16_t* out;
+  int32_t heads;
+  int32_t q_rows;
+  int32_t n_nodes;
+  int32_t pad;
+  AttnNode nodes[WAVE_MAX_NODES];
+  int32_t block0[WAVE_MAX_NODES + 1];  // first CTA of each node (nodes without ranges: none)
+};
+constexpr int kCombineRowsPerCta = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kCombineRowsPerCta)
+    attn_combine_kernel(const __grid_constant__ CombineParams p) {
+  constexpr int V = D / 32;  // O values per lane
+  constexpr int kCtasPerTile = 128 / kCombineRowsPerCta;
+  int n = 0;
+  while (n + 1 < p.n_nodes && (int)blockIdx.x >= p.block0[n + 1]) ++n;
+  const AttnNode& nd = p.nodes[n];
+  const int j = (blockIdx.x - p.block0[n]) / kCtasPerTile;
+  const int head = j / nd.n_qtiles, qt = j - head * nd.n_qtiles;
+  const int pair = qt >> 1, w = qt & 1, S = nd.n_splits;
+  const int64_t item_base = nd.item0 + (int64_t)(head * nd.n_pairs + pair) * S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {
+    const int r = ((blockIdx.x - p.block0[n]) % kCtasPerTile) * kCombineRowsPerCta + warp;
+    const int q_local = qt * 128 + r;
+    if (q_local >= p.q_rows) return;
+    float m = -INFINITY, l = 0.f;
+    if (lane < S) {
+      const float2 ml = reinterpret_cast<const float2*>(p.part_ml)[((item_base + lane) * 2 + w) * 128 + r];
+      m = ml.x;
+      l = ml.y;
+    }
+    float mx = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float e = lane < S ? exp2f(m - mx) : 0.f;
+    float den = e * l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < S; ++sp) {
+      const float es = __shfl_sync(0xffffffffu, e, sp);
+      const float* po = p.part_o + (((item_base + sp) * 2 + w) * 128 + r) * D + lane * V;
+      if constexpr (V == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(po);
+        acc[0] += es * v.x; acc[1] += es * v.y; acc[2] += es * v.z; acc[3] += es * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(po);
+        acc[0] += es * v.x; acc[1] += es * v.y;
+      }
+    }
+    const float inv = 1.f / den;
+    uint16_t* dst = p.out + ((int64_t)(nd.q_row0 + q_local) * p.heads + head) * D + lane * V;
+    if constexpr (V == 4) {
+      *reinterpret_cast<uint2*>(dst) =
+          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+  }
+}
+
 template <int D>
 int launch(const AttnParams& prm, int grid, cudaStream_t stream) {
   static std::once_flag once;
@@ -671,8 +779,30 @@ namespace {
 
 // One round of attention with the work-queue counter at `counter` (a device
 // int32 that this call sets to zero on `stream` before the launch).
+// Key ranges per (node, head, pair) for a call: `splits` >= 1 as asked; 0 =
+// none when the round already has a wave of items for the SMs (the dynamic
+// longest-first queue balances those), else enough for about two waves; at
+// most the node's pages and kMaxSplits.
+constexpr int kMaxSplits = 32;
+int choose_splits(const wave_kv* kv, int32_t n_active, int32_t splits) {
+  if (splits > 0) return std::min(splits, kMaxSplits);
+  const int T = kv->cfg.tokens_per_chunk, H = kv->cfg.heads;
+  const int64_t items = (int64_t)n_active * H * (((T + 127) / 128 + 1) / 2);
+  if (items >= kv->num_sms) return 1;
+  const int64_t want = 2LL * kv->num_sms;
+  return (int)std::min<int64_t>(kMaxSplits, (want + items - 1) / items);
+}
+
+// Bytes of workspace a split call needs: per work item and query tile, 128
+// rows of d fp32 O values and an fp32 (max, sum) pair.
+uint64_t split_workspace_bytes(const wave_kv* kv, int64_t n_items) {
+  return (uint64_t)n_items * 2 * 128 * ((uint64_t)kv->cfg.head_dim + 2) * sizeof(float);
+}
+
 int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
-                    const void* Q, void* O, void* stream, int32_t* counter) {
+                    const void* Q, void* O, void* stream, int32_t* counter, int32_t splits = 1,
+                    void* workspace = nullptr, uint64_t workspace_bytes = 0,
+                    uint64_t* bytes_needed = nullptr) {
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
   if (int rc = check_current_device(kv)) return rc;
@@ -681,7 +811,8 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
   if (n_active == 0) return WAVE_OK;
   if (n_active > WAVE_MAX_NODES)
     return fail(WAVE_ERR_CAPACITY, "%d active nodes exceed %d", n_active, WAVE_MAX_NODES);
-  if (!Q || !O || ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15))
+  if (!bytes_needed &&
+      (!Q || !O || ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) & 15)))
     return fail(WAVE_ERR_ARG, "Q and O must be non-NULL and 16-byte aligned");
   std::vector<int32_t> rows, offs;
   int rc = build_rows(kv, active, n_active, policy, rows, offs);
@@ -696,6 +827,32 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
 
   static thread_local AttnParams prm;
   std::memset(&prm, 0, offsetof(AttnParams, pages));
+  // Nodes in longest-key-list-first order, each with its key ranges.
+  const int n_qtiles = (T + 127) / 128;
+  const int n_pairs = (n_qtiles + 1) / 2;
+  std::vector<int> order(n_active);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return offs[a + 1] - offs[a] > offs[b + 1] - offs[b];
+  });
+  int64_t n_items = 0;
+  bool any_split = false;
+  for (int k = 0; k < n_active; ++k) {
+    const int i = order[k];
+    const int ns = std::max(1, std::min<int>(splits, offs[i + 1] - offs[i]));
+    any_split |= ns > 1;
+    n_items += (int64_t)H * n_pairs * ns;
+  }
+  if (n_items >= (1LL << 30)) return fail(WAVE_ERR_CAPACITY, "too many work items");
+  const uint64_t need = any_split ? split_workspace_bytes(kv, n_items) : 0;
+  if (bytes_needed) {
+    *bytes_needed = need;
+    return WAVE_OK;
+  }
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   (reinterpret_cast<uintptr_t>(workspace) & 15)))
+    return fail(WAVE_ERR_ARG, "split key ranges need a 16-byte aligned workspace of %llu bytes "
+                "(got %llu)", (unsigned long long)need, (unsigned long long)workspace_bytes);
   auto encode = tensor_map_encoder();
   if (!encode) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)n_active * T};
@@ -719,13 +876,6 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
 
   // Longest key list first (ties keep list order): a static round-robin of
   // items over persistent CTAs then approximates longest-processing-time order.
-  std::vector<int> order(n_active);
-  std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-    return offs[a + 1] - offs[a] > offs[b + 1] - offs[b];
-  });
-  const int n_qtiles = (T + 127) / 128;
-  const int n_pairs = (n_qtiles + 1) / 2;
   int32_t item0 = 0, w = 0;
   for (int k = 0; k < n_active; ++k) {
     const int i = order[k];
@@ -736,16 +886,45 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
     nd.item0 = item0;
     nd.n_pairs = n_pairs;
     nd.n_qtiles = n_qtiles;
+    nd.n_splits = std::max(1, std::min<int>(splits, nd.n_pages));
     for (int32_t rr = offs[i]; rr < offs[i + 1]; ++rr)
       prm.pages[w++] = (uint32_t)rows[2 * rr] | ((uint32_t)(rows[2 * rr + 1] - 1) << 25);
-    item0 += H * n_pairs;
+    item0 += H * n_pairs * nd.n_splits;
   }
   prm.n_items = item0;
+  if (any_split) {
+    prm.part_o = static_cast<float*>(workspace);
+    prm.part_ml = prm.part_o + (int64_t)item0 * 2 * 128 * D;
+  }
   const int grid = std::min(prm.n_items, kv->num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(prm.counter, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "cudaMemsetAsync(work counter): %s", cudaGetErrorString(e));
-  return D == 128 ? launch<128>(prm, grid, s) : launch<64>(prm, grid, s);
+  rc = D == 128 ? launch<128>(prm, grid, s) : launch<64>(prm, grid, s);
+  if (rc || !any_split) return rc;
+  // Combine the key ranges of every split node into O.
+  static thread_local CombineParams cp;
+  std::memset(&cp, 0, sizeof(cp));
+  cp.part_o = prm.part_o;
+  cp.part_ml = prm.part_ml;
+  cp.out = prm.out;
+  cp.heads = H;
+  cp.q_rows = T;
+  cp.n_nodes = n_active;
+  int32_t blocks = 0;
+  for (int k = 0; k < n_active; ++k) {
+    cp.nodes[k] = prm.nodes[k];
+    cp.block0[k] = blocks;
+    if (prm.nodes[k].n_splits > 1) blocks += H * n_qtiles * (128 / kCombineRowsPerCta);
+  }
+  cp.block0[n_active] = blocks;
+  if (D == 128)
+    attn_combine_kernel<128><<<blocks, 32 * kCombineRowsPerCta, 0, s>>>(cp);
+  else
+    attn_combine_kernel<64><<<blocks, 32 * kCombineRowsPerCta, 0, s>>>(cp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "attn_combine_kernel launch: %s", cudaGetErrorString(e));
+  return WAVE_OK;
 }
 
 }  // namespace
@@ -759,6 +938,33 @@ extern "C" int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_a
   int32_t* counter =
       reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
   return round_attn_impl(kv, active, n_active, policy, Q, O, stream, counter);
+}
+
+extern "C" int wave_round_attn_split_workspace(wave_kv* kv, const wave_node* active,
+                                               int32_t n_active, int32_t policy, int32_t splits,
+                                               uint64_t* bytes, int32_t* splits_used) {
+  clear_error();
+  if (!kv || !bytes) return fail(WAVE_ERR_ARG, "NULL argument");
+  if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
+  if (splits < 0) return fail(WAVE_ERR_ARG, "splits must be >= 0, got %d", splits);
+  const int ns = choose_splits(kv, n_active, splits);
+  if (splits_used) *splits_used = ns;
+  int32_t* counter = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
+  return round_attn_impl(kv, active, n_active, policy, nullptr, nullptr, nullptr, counter, ns,
+                         nullptr, 0, bytes);
+}
+
+extern "C" int wave_round_attn_split(wave_kv* kv, const wave_node* active, int32_t n_active,
+                                     int32_t policy, int32_t splits, const void* Q, void* O,
+                                     void* workspace, uint64_t workspace_bytes, void* stream) {
+  clear_error();
+  if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
+  if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL)");
+  if (splits < 0) return fail(WAVE_ERR_ARG, "splits must be >= 0, got %d", splits);
+  int32_t* counter =
+      reinterpret_cast<int32_t*>(static_cast<uint8_t*>(kv->cfg.pool) + kCounterOffset);
+  return round_attn_impl(kv, active, n_active, policy, Q, O, stream, counter,
+                         choose_splits(kv, n_active, splits), workspace, workspace_bytes);
 }
 
 // ----------------------------------------------------------------------------

@@ -103,9 +103,23 @@ struct GemmParams {
 };
 static_assert(sizeof(GemmParams) <= 32760, "kernel parameter space is 32 KB");
 
+// GELU, tanh form, through 0.5 (1 + tanh u) = 1 / (1 + e^(-2u)): one
+// exponential and one division on the special-function unit, with relative
+// accuracy everywhere (the tail where 1 + tanh u is tiny included).
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
-  return 0.5f * x * (1.f + tanhf(u));
+  return __fdividef(x, 1.f + __expf(-2.f * u));
+}
+
+// sin and cos of a rotary angle: reduced to [-pi, pi] by subtracting the
+// nearest multiple of 2 pi (Cody-Waite: 2 pi split into 6.28125, exact in a
+// few bits, plus the remainder, so k * 6.28125 is exact for the k that occur),
+// then the special-function unit's sin/cos, accurate to ~4e-7 on [-pi, pi].
+__device__ __forceinline__ void rope_sincos(float a, float* sn, float* cs) {
+  const float k = rintf(a * 0.15915494309189535f);
+  float r = fmaf(-k, 6.28125f, a);
+  r = fmaf(-k, 1.9353071795864769e-3f, r);
+  __sincosf(r, sn, cs);
 }
 
 __device__ __forceinline__ int64_t a_row0(const GemmParams& p, int mt) {
@@ -298,7 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int j = 0; j < 16; ++j) {
                 const int pr = 16 * c + j;
                 float sn, cs;
-                sincosf(pos[p.rope_axis[pr]] * p.rope_theta[pr], &sn, &cs);
+                rope_sincos(pos[p.rope_axis[pr]] * p.rope_theta[pr], &sn, &cs);
                 const float a = f[2 * j], b = f[2 * j + 1];
                 f[2 * j] = a * cs - b * sn;
                 f[2 * j + 1] = a * sn + b * cs;

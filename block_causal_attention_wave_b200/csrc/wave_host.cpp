@@ -11,6 +11,7 @@
 #include <cstring>
 #include <set>
 #include <string>
+#include <tuple>
 
 #include "wave_internal.h"
 
@@ -418,6 +419,90 @@ int wave_schedule_last_read(int32_t B, int32_t K, int32_t policy, int32_t window
         rnd[(size_t)nd.chunk * (K + 1) + nd.level] < 0)
       return fail(WAVE_ERR_ARG, "(%d, %d) is not a node of this schedule", nd.chunk, nd.level);
     last_round[i] = last[(size_t)nd.chunk * (K + 1) + nd.level];
+  }
+  return WAVE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Wave Parallelism (Wave Forcing page, "Key Findings"; "Wave Forcing Targets
+// Near-Light-Speed Video Streaming Generation": one-way K/V communication
+// between full-model replicas): node (c, l) runs on rank l mod N; the entry a
+// node produces is pushed in its own round to every other rank that runs a
+// node reading it.
+
+extern "C" {
+
+int wave_wp_transfers(int32_t B, int32_t K, int32_t policy, int32_t window, int32_t n_ranks,
+                      int32_t round, wave_transfer* out, int32_t cap, int32_t* n) {
+  using namespace wavei;
+  clear_error();
+  if (!n || n_ranks < 1) return fail(WAVE_ERR_ARG, "need n_ranks >= 1 and a count pointer");
+  std::vector<int32_t> rnd;
+  int32_t nn = 0, nr = 0;
+  int rc = compute_rounds(B, K, policy, window, rnd, &nn, &nr);
+  if (rc) return rc;
+  if (round < 0 || round >= nr) return fail(WAVE_ERR_ARG, "round %d outside 0..%d", round, nr - 1);
+  // Ranks reading each entry: the producer's own, plus those of its readers.
+  std::vector<std::set<int32_t>> dst((size_t)B * (K + 1));
+  for (int c = 0; c < B; ++c)
+    for (int l = 0; l <= K; ++l) {
+      if (rnd[(size_t)c * (K + 1) + l] < 0) continue;
+      const int span = window <= 0 ? c : std::min<int>(c, window);
+      for (int r = 1; r <= span; ++r)
+        dst[(size_t)(c - r) * (K + 1) + phi(policy, l, r)].insert(l % n_ranks);
+    }
+  std::vector<wave_transfer> t;
+  for (int c = 0; c < B; ++c)
+    for (int l = 0; l <= K; ++l) {
+      if (rnd[(size_t)c * (K + 1) + l] != round) continue;
+      const int32_t src = l % n_ranks;
+      for (int32_t d : dst[(size_t)c * (K + 1) + l])
+        if (d != src) t.push_back(wave_transfer{c, l, src, d});
+    }
+  // Sorted by (chunk, level, src, dst): the order every rank walks them in.
+  std::sort(t.begin(), t.end(), [](const wave_transfer& a, const wave_transfer& b) {
+    return std::make_tuple(a.chunk, a.level, a.src, a.dst) <
+           std::make_tuple(b.chunk, b.level, b.src, b.dst);
+  });
+  *n = (int32_t)t.size();
+  if (*n > cap || (*n > 0 && !out))
+    return fail(WAVE_ERR_CAPACITY, "round %d has %d transfers, capacity %d", round, *n, cap);
+  if (*n > 0) std::memcpy(out, t.data(), t.size() * sizeof(wave_transfer));
+  return WAVE_OK;
+}
+
+int wave_wp_rank_last_read(int32_t B, int32_t K, int32_t policy, int32_t window, int32_t n_ranks,
+                           int32_t rank, const wave_node* entries, int32_t n,
+                           int32_t* last_round) {
+  using namespace wavei;
+  clear_error();
+  if (n_ranks < 1 || rank < 0 || rank >= n_ranks || n < 0 || (n > 0 && (!entries || !last_round)))
+    return fail(WAVE_ERR_ARG, "bad arguments");
+  std::vector<int32_t> rnd;
+  int32_t nn = 0, nr = 0;
+  int rc = compute_rounds(B, K, policy, window, rnd, &nn, &nr);
+  if (rc) return rc;
+  std::vector<int32_t> last((size_t)B * (K + 1), -1);
+  for (int c = 0; c < B; ++c)
+    for (int l = 0; l <= K; ++l) {
+      const int32_t t = rnd[(size_t)c * (K + 1) + l];
+      if (t < 0 || l % n_ranks != rank) continue;
+      int32_t& own = last[(size_t)c * (K + 1) + l];
+      own = std::max(own, t);
+      const int span = window <= 0 ? c : std::min<int>(c, window);
+      for (int r = 1; r <= span; ++r) {
+        int32_t& e = last[(size_t)(c - r) * (K + 1) + phi(policy, l, r)];
+        e = std::max(e, t);
+      }
+    }
+  for (int32_t i = 0; i < n; ++i) {
+    const wave_node& e = entries[i];
+    if (e.chunk < 0 || e.chunk >= B || e.level < 0 || e.level > K ||
+        last[(size_t)e.chunk * (K + 1) + e.level] < 0)
+      return fail(WAVE_ERR_ARG, "rank %d holds no entry (%d, %d)", rank, e.chunk, e.level);
+    last_round[i] = last[(size_t)e.chunk * (K + 1) + e.level];
   }
   return WAVE_OK;
 }

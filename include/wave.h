@@ -257,6 +257,35 @@ int wave_gather_table(const wave_kv* kv, const wave_node* active, int32_t n_acti
 int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
                     const void* Q, void* O, void* stream);
 
+/* wave_round_attn with each node's key list cut into key ranges (split-KV),
+ * for rounds with too few (node, head, query-tile pair) work items to fill
+ * the GPU -- short query blocks over long K/V, e.g. one Wan-Streamer unit of
+ * 984 tokens over 32 units of history and a 512-token prefix ([WS] abstract,
+ * glossary "K/V cache", "streaming unit"). Every (node, head, pair) item
+ * becomes min(splits, node pages) items over consecutive page ranges; each
+ * writes its unnormalised O rows and their (running max, sum) to
+ * `workspace`, and a second kernel on `stream` combines them:
+ * O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s -- the same
+ * softmax(Q K^T / sqrt(d)) V as wave_round_attn, up to rounding.
+ * splits: >= 1 ranges per item (at most 32), or 0 = enough to give the GPU
+ * about two waves of items (1 when the round already has a wave of them).
+ * workspace: device buffer, 16-byte aligned, at least the bytes
+ * wave_round_attn_split_workspace reports for the same arguments (none is
+ * needed when no node is split); caller-owned, its contents are scratch.
+ * Other arguments, layouts, limits and errors as wave_round_attn; ARG also
+ * for a missing or too small workspace. */
+int wave_round_attn_split(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
+                          int32_t splits, const void* Q, void* O, void* workspace,
+                          uint64_t workspace_bytes, void* stream);
+
+/* Workspace bytes wave_round_attn_split needs for these arguments (0 if no
+ * node ends up split) and, in *splits_used (may be NULL), the ranges per item
+ * it will use (splits = 0 resolved). Host only. Errors: as wave_round_attn's
+ * table checks (ARG, MISSING_KV, CAPACITY). */
+int wave_round_attn_split_workspace(wave_kv* kv, const wave_node* active, int32_t n_active,
+                                    int32_t policy, int32_t splits, uint64_t* bytes,
+                                    int32_t* splits_used);
+
 /* wave_round_attn without per-call scratch from the caller. The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory for the library while they run -- e.g. code inside CUDA stream
@@ -322,6 +351,38 @@ int wave_schedule(int32_t B, int32_t K, int32_t policy, int32_t window, wave_nod
  * Errors: ARG (bad sizes, or a node that is not in the schedule). */
 int wave_schedule_last_read(int32_t B, int32_t K, int32_t policy, int32_t window,
                             const wave_node* nodes, int32_t n, int32_t* last_round);
+
+/* ---- Wave Parallelism: one node per GPU, one-way K/V pushes ----------------
+ * [WF] "Key Findings" (full-model replicas, early K/V delivery) and
+ * "Wave Forcing Targets Near-Light-Speed Video Streaming Generation"
+ * (aipulsen.com): Wave Parallelism with one-way key-value communication. The
+ * pages give no placement or protocol; the reading implemented here: node
+ * (c, l) runs on rank l mod n_ranks (with K + 1 ranks, one per denoising
+ * level); the entry E(c, l) a node produces is pushed, in the node's own
+ * round and before that round's attention, from its rank to every other rank
+ * that runs a node reading it. Under the progressive policy pushes only go
+ * from a cleaner level's rank to a noisier one; under same-level with a rank
+ * per level there are none. Each rank keeps its own pool: per round it
+ * appends the entries its nodes produce (node order), then takes pages for
+ * the entries it receives (ascending (chunk, level)) and receives their page
+ * bytes; it releases an entry after wave_wp_rank_last_read's round. */
+typedef struct {
+  int32_t chunk, level; /* the entry E(chunk, level)                           */
+  int32_t src, dst;     /* producer's rank -> a reader's rank (src != dst)      */
+} wave_transfer;
+
+/* Pushes of `round` of the (B, K, policy, window) schedule on n_ranks ranks,
+ * sorted by (chunk, level, src, dst). `cap` = capacity of out; *n = count.
+ * Host only. Errors: ARG, CAPACITY (*n = entries needed). */
+int wave_wp_transfers(int32_t B, int32_t K, int32_t policy, int32_t window, int32_t n_ranks,
+                      int32_t round, wave_transfer* out, int32_t cap, int32_t* n);
+
+/* For each entry, the last round in which a node that runs on `rank` reads it
+ * (the round after which that rank releases it). Host only. Errors: ARG (an
+ * entry the rank never holds). */
+int wave_wp_rank_last_read(int32_t B, int32_t K, int32_t policy, int32_t window, int32_t n_ranks,
+                           int32_t rank, const wave_node* entries, int32_t n,
+                           int32_t* last_round);
 
 /* Static name of a status code. */
 const char* wave_strerror(int code);
