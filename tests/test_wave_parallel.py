@@ -87,7 +87,7 @@ def _worker(rank, world, port, cfg, out):
 ])
 def test_wave_parallel_rollout_over_gloo(cfg, world):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, cfg, out), nprocs=world, join=True)
         assert dict(out) == {r: "ok" for r in range(world)}
