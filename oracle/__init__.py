@@ -25,6 +25,8 @@ What it computes, each part written as the plain definition from the pages:
                                (frame, row, column), out-projection and
                                tanh-GELU MLP with residuals, bf16 storage
                                between kernels (readings stated there).
+* ``quant``                 -- FP8 (E4M3) K/V pages with per-(page, head)
+                               scales and their bf16 read-back.
 * ``parallel``              -- Wave Parallelism host logic: node placement on
                                ranks, one-way K/V pushes per round, and each
                                rank's page tables.
@@ -35,4 +37,4 @@ torch's CPU attention, exhaustive search). Absolute attention values printed by
 the pages: none exist, so that part is "parity unpinned" against the pages and
 pinned only by the mathematics.
 """
-from . import policy, schedule, cache, attention, projection, block, parallel  # noqa: F401
+from . import policy, schedule, cache, attention, projection, block, parallel, quant  # noqa: F401
