@@ -332,6 +332,35 @@ def run_gpu(args):
     value = ws * flops * K / (ms * 1e-3) / 1e12
     attn_avg = sum(attn_ms) / len(attn_ms)
 
+    # ---- the round's 4 update nodes alone (the refresh node's queries left out):
+    # the 2.9605-TFLOP headline of the round, beside the 5-node figure above.
+    upd_only = [n for n in active if n[1] > 0]
+    updates = None
+    if len(upd_only) < len(active):
+        idx = [active.index(n) for n in upd_only]
+        T = wl.tokens
+        q_u = torch.cat([dq[i * T:(i + 1) * T] for i in idx])
+        o_u = torch.empty_like(q_u)
+        kv.append_batch(active, dk, dv, stream)
+        u_table = kv.gather_table(upd_only, POLICY)
+        u_flops = sum(4 * T * sum(v for _, v in rows) * wl.heads * wl.head_dim for rows in u_table)
+        for _ in range(3):
+            kv.round_attn(upd_only, POLICY, q_u, o_u, stream)
+        ua, ub = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e6))
+        ua.record(stream)
+        for _ in range(10):
+            kv.round_attn(upd_only, POLICY, q_u, o_u, stream)
+        ub.record(stream)
+        torch.cuda.synchronize()
+        for n in active:
+            kv.release(*n)
+        u_ms = ua.elapsed_time(ub) / 10
+        updates = {"nodes": [list(n) for n in upd_only], "flops_per_launch": u_flops,
+                   "avg_launch_ms": round(u_ms, 4),
+                   "achieved": round(u_flops / (u_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                   "chunk_updates_per_s": round(len(upd_only) / (u_ms * 1e-3), 2)}
+
     # ---- the batched append launch (HBM roofline context): events around it in
     # every timed step. The host runs ahead of the GPU during each attention
     # launch, so these events see the kernel, not the host's enqueue time; the
@@ -386,6 +415,13 @@ def run_gpu(args):
     block = None
     if spec.key == DEFAULT_WORKLOAD and not args.no_block:
         block = block_round(wave, kv, wl, active, stream, args)
+
+    # ---- FP8 (E4M3) pages: the same round over an FP8 pool holding the round's
+    # key lists (history appended once, quantised); per step the round's pages
+    # are expanded to bf16 staging in the workspace, then the attention runs.
+    fp8 = None
+    if spec.key == DEFAULT_WORKLOAD and not args.no_block:
+        fp8 = fp8_round(wave, wl, rd, active, dq, stream, flops)
 
     # ---- split-KV attention (key lists cut into ranges, partials combined):
     # the same round with the automatic range count, and a round of a single
@@ -487,9 +523,11 @@ def run_gpu(args):
                    "frac": round(append_bytes / (append_ms * 1e-3) / 1e9 /
                                  peaks["hbm_gbs"], 4)},
         "gpu_launches": K * 2,
+        "updates_only": updates,
         "projection": proj,
         "block": block,
         "split_kv": split,
+        "fp8_pages": fp8,
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and spec.key == DEFAULT_WORKLOAD:
@@ -499,6 +537,54 @@ def run_gpu(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def fp8_round(wave, wl, rd, active, dq, stream, flops):
+    """Attention of the round over an FP8 pool: expand + attention per step."""
+    import torch
+    ents = set()
+    table_nodes = active
+    pb8 = wave.KVCache.page_bytes(wl.heads, wl.head_dim, wave.KV_FP8_E4M3)
+    pb16 = wave.KVCache.page_bytes(wl.heads, wl.head_dim)
+    pages = 1000
+    pool = torch.zeros(4096 + 256 + pages * (pb8 + 2 * wl.heads * 4), dtype=torch.uint8,
+                       device="cuda")
+    kv8 = wave.KVCache(wl.heads, wl.head_dim, wl.tokens, wl.levels, wl.window, wl.prefix,
+                       pool=pool, kv_format=wave.KV_FP8_E4M3)
+    # every entry the round's nodes read: history from earlier rounds, then the round's own
+    last = rd.last
+    for t in range(rd.spec.round + 1):
+        for n in rd.rounds[t]:
+            if last[tuple(n)] >= rd.spec.round:
+                ents.add(tuple(n))
+    for e in sorted(ents):
+        kv8.append(e[0], e[1],
+                   _bits_to_dev(wi.node_tensor("k", e[0], e[1], wl.tokens, wl.heads, wl.head_dim,
+                                               wl.scale)),
+                   _bits_to_dev(wi.node_tensor("v", e[0], e[1], wl.tokens, wl.heads, wl.head_dim,
+                                               wl.scale)), stream)
+    nbytes, _ = kv8.split_workspace(table_nodes, POLICY, 1)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(dq)
+    for _ in range(3):
+        kv8.round_attn_split(table_nodes, POLICY, dq, o, ws, 1, stream)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    torch.cuda._sleep(int(2e6))
+    ev[0].record(stream)
+    for _ in range(10):
+        kv8.round_attn_split(table_nodes, POLICY, dq, o, ws, 1, stream)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    kv8.status(stream)
+    ms = ev[0].elapsed_time(ev[1]) / 10
+    n_pages = len({p for rows in kv8.gather_table(table_nodes, POLICY) for p, _ in rows})
+    return {"what": "attention of the round over an FP8 (E4M3, per-(page, head) scale) pool: "
+                    "the round's pages expanded to bf16 staging, then the attention kernel",
+            "entry_bytes_bf16": (wl.tokens + 127) // 128 * pb16,
+            "entry_bytes_fp8": (wl.tokens + 127) // 128 * (pb8 + 2 * wl.heads * 4),
+            "round_pages": n_pages, "staging_bytes": nbytes,
+            "ms": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
 
 
 def split_rounds(wave, kv, wl, active, dq, do, stream, flops):
@@ -676,16 +762,35 @@ def _cores():
         return os.cpu_count()
 
 
+# Query rows per node in one oracle sample: the same sample for the CPU-baseline
+# leg (repeated for about --cpu-seconds) and for each step of the reference arm.
+ORACLE_SAMPLE_ROWS = 32
+
+
 def cpu_baseline(target_s=10.0):
     active, entries, qs = _oracle_round()
     _oracle_sample(active, entries, qs, 4)  # first touch of the float64 inputs
-    dt, _, _ = _oracle_sample(active, entries, qs, 16)
-    n_rows = int(min(1024, max(16, 16 * target_s / max(dt, 1e-3))))
-    dt, flops, nr = _oracle_sample(active, entries, qs, n_rows)
-    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": _cores(),
-            "kind": "oracle",
-            "sample": f"{nr} of 4680 query rows of each of the 5 nodes, all 12 heads, full key "
-                      f"lists ({flops / 1e9:.1f} GFLOP in {dt:.2f} s, float64 numpy)"}
+    total, flops, reps, nr = 0.0, 0, 0, 0
+    while total < target_s or reps < 1:
+        dt, f, nr = _oracle_sample(active, entries, qs, ORACLE_SAMPLE_ROWS)
+        total += dt
+        flops += f
+        reps += 1
+    out = {"value": round(flops / total / 1e12, 6), "unit": UNIT, "cores": _cores(),
+           "kind": "oracle",
+           "sample": f"{reps} x {nr} of 4680 query rows of each of the 5 nodes, all 12 heads, "
+                     f"full key lists ({flops / 1e9:.1f} GFLOP in {total:.2f} s, float64 numpy); "
+                     "the reference arm times the same sample per step"}
+    try:  # the same sample on one core
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(limits=1):
+            dt1, f1, _ = _oracle_sample(active, entries, qs, ORACLE_SAMPLE_ROWS)
+        out["value_1core"] = round(f1 / dt1 / 1e12, 6)
+        out["sample_1core"] = f"one sample ({f1 / 1e9:.1f} GFLOP in {dt1:.2f} s) on 1 thread"
+    except Exception as e:  # threadpoolctl missing: no 1-core figure
+        out["value_1core"] = None
+        out["sample_1core"] = f"not measured: {type(e).__name__}"
+    return out
 
 
 def run_reference(args):
@@ -693,7 +798,7 @@ def run_reference(args):
     if rank != 0:
         return
     active, entries, qs = _oracle_round()
-    n_rows = 24
+    n_rows = ORACLE_SAMPLE_ROWS
     for _ in range(args.warmup):
         _oracle_sample(active, entries, qs, n_rows)
     times, flops = [], 0

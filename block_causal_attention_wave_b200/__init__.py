@@ -8,5 +8,5 @@ launch. This package is its thin ctypes binding.
 from ._binding import (  # noqa: F401
     KVCache, Node, WaveError, load, schedule, last_read_rounds, exported_symbols,
     wp_transfers, wp_rank_last_read,
-    POLICIES, PAGE_TOKENS, ACT_NONE, ACT_GELU_TANH, PREFIX_CHUNK, MAX_NODES, MAX_PAGES_PER_ROUND, LIB_PATH,
+    POLICIES, PAGE_TOKENS, ACT_NONE, ACT_GELU_TANH, KV_BF16, KV_FP8_E4M3, PREFIX_CHUNK, MAX_NODES, MAX_PAGES_PER_ROUND, LIB_PATH,
 )

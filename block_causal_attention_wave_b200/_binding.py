@@ -41,6 +41,7 @@ class Rope(ctypes.Structure):
 
 
 ACT_NONE, ACT_GELU_TANH = 0, 1
+KV_BF16, KV_FP8_E4M3 = 0, 1
 
 
 class Transfer(ctypes.Structure):
@@ -52,12 +53,14 @@ class KVConfig(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("tokens_per_chunk", ctypes.c_int32), ("num_levels", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("prefix_tokens", ctypes.c_int32),
-                ("pool", ctypes.c_void_p), ("pool_bytes", ctypes.c_uint64)]
+                ("pool", ctypes.c_void_p), ("pool_bytes", ctypes.c_uint64),
+                ("kv_format", ctypes.c_int32)]
 
 
 _SIGS = {
     "wave_kv_create": (ctypes.c_int, [ctypes.POINTER(KVConfig), ctypes.POINTER(ctypes.c_void_p)]),
     "wave_kv_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "wave_kv_scale_offset": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)]),
     "wave_kv_pool_layout": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64),
                                            ctypes.POINTER(ctypes.c_int64),
                                            ctypes.POINTER(ctypes.c_int32)]),
@@ -243,7 +246,7 @@ class KVCache:
     """
 
     def __init__(self, heads, head_dim, tokens_per_chunk, num_levels, window=0,
-                 prefix_tokens=0, pool=None, pool_bytes=None):
+                 prefix_tokens=0, pool=None, pool_bytes=None, kv_format=0):
         self.lib = load()
         self.heads, self.head_dim = heads, head_dim
         self.tokens, self.levels = tokens_per_chunk, num_levels
@@ -255,14 +258,22 @@ class KVCache:
         else:
             ptr = None
         cfg = KVConfig(heads, head_dim, tokens_per_chunk, num_levels, window, prefix_tokens,
-                       ptr, int(pool_bytes))
+                       ptr, int(pool_bytes), int(kv_format))
+        self.kv_format = int(kv_format)
         h = ctypes.c_void_p()
         _check(self.lib.wave_kv_create(ctypes.byref(cfg), ctypes.byref(h)))
         self.h = h
 
     @staticmethod
-    def page_bytes(heads, head_dim) -> int:
-        return 2 * heads * PAGE_TOKENS * head_dim * 2
+    def page_bytes(heads, head_dim, kv_format=0) -> int:
+        """Bytes of one page (an FP8 pool also keeps 2 H float32 scales per page)."""
+        return 2 * heads * PAGE_TOKENS * head_dim * (1 if kv_format == KV_FP8_E4M3 else 2)
+
+    def scale_offset(self) -> int:
+        """Byte offset of an FP8 pool's scale table, float32 [max_pages][2][H]."""
+        off = ctypes.c_int64()
+        _check(self.lib.wave_kv_scale_offset(self.h, ctypes.byref(off)))
+        return off.value
 
     def close(self):
         if getattr(self, "h", None):

@@ -41,6 +41,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <numeric>
 #include <vector>
@@ -844,15 +845,26 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
     n_items += (int64_t)H * n_pairs * ns;
   }
   if (n_items >= (1LL << 30)) return fail(WAVE_ERR_CAPACITY, "too many work items");
-  const uint64_t need = any_split ? split_workspace_bytes(kv, n_items) : 0;
+  // FP8 pools: the round's distinct pages are expanded to bf16 staging pages
+  // (slot = order of first use) at the start of the workspace.
+  std::vector<int32_t> slot_page;
+  std::map<int32_t, int32_t> slot_of;
+  if (kv->fp8) {
+    for (int64_t rr = 0; rr < n_rows; ++rr)
+      if (slot_of.emplace(rows[2 * rr], (int32_t)slot_page.size()).second)
+        slot_page.push_back(rows[2 * rr]);
+  }
+  const uint64_t staging = ((uint64_t)slot_page.size() * bf16_page_bytes(kv) + 255) / 256 * 256;
+  const uint64_t need = staging + (any_split ? split_workspace_bytes(kv, n_items) : 0);
   if (bytes_needed) {
     *bytes_needed = need;
     return WAVE_OK;
   }
   if (need > 0 && (!workspace || workspace_bytes < need ||
-                   (reinterpret_cast<uintptr_t>(workspace) & 15)))
-    return fail(WAVE_ERR_ARG, "split key ranges need a 16-byte aligned workspace of %llu bytes "
-                "(got %llu)", (unsigned long long)need, (unsigned long long)workspace_bytes);
+                   (reinterpret_cast<uintptr_t>(workspace) & 255)))
+    return fail(WAVE_ERR_ARG, "%s need a 256-byte aligned workspace of %llu bytes (got %llu; "
+                "use wave_round_attn_split)", kv->fp8 ? "FP8 pages" : "split key ranges",
+                (unsigned long long)need, (unsigned long long)workspace_bytes);
   auto encode = tensor_map_encoder();
   if (!encode) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)n_active * T};
@@ -863,7 +875,19 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled(Q) failed: %d", (int)r);
-  prm.tm_kv = kv->tm_kv;
+  if (kv->fp8) {
+    cuuint64_t sd[2] = {(cuuint64_t)D, (cuuint64_t)slot_page.size() * 2 * H * kPageTokens};
+    cuuint64_t ss[1] = {(cuuint64_t)D * 2};
+    cuuint32_t sb[2] = {64, 128};
+    cuuint32_t se[2] = {1, 1};
+    r = encode(&prm.tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, sd, ss, sb, se,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(WAVE_ERR_CUDA, "cuTensorMapEncodeTiled(staging) failed: %d", (int)r);
+  } else {
+    prm.tm_kv = kv->tm_kv;
+  }
   prm.out = static_cast<uint16_t*>(O);
   prm.status = static_cast<int32_t*>(kv->cfg.pool);
   prm.counter = counter;
@@ -887,17 +911,23 @@ int round_attn_impl(wave_kv* kv, const wave_node* active, int32_t n_active, int3
     nd.n_pairs = n_pairs;
     nd.n_qtiles = n_qtiles;
     nd.n_splits = std::max(1, std::min<int>(splits, nd.n_pages));
-    for (int32_t rr = offs[i]; rr < offs[i + 1]; ++rr)
-      prm.pages[w++] = (uint32_t)rows[2 * rr] | ((uint32_t)(rows[2 * rr + 1] - 1) << 25);
+    for (int32_t rr = offs[i]; rr < offs[i + 1]; ++rr) {
+      const int32_t pg = kv->fp8 ? slot_of[rows[2 * rr]] : rows[2 * rr];
+      prm.pages[w++] = (uint32_t)pg | ((uint32_t)(rows[2 * rr + 1] - 1) << 25);
+    }
     item0 += H * n_pairs * nd.n_splits;
   }
   prm.n_items = item0;
   if (any_split) {
-    prm.part_o = static_cast<float*>(workspace);
+    prm.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + staging);
     prm.part_ml = prm.part_o + (int64_t)item0 * 2 * 128 * D;
   }
   const int grid = std::min(prm.n_items, kv->num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (kv->fp8) {
+    rc = launch_fp8_expand(kv, (int32_t)slot_page.size(), slot_page.data(), workspace, s);
+    if (rc) return rc;
+  }
   cudaError_t e = cudaMemsetAsync(prm.counter, 0, sizeof(int32_t), s);
   if (e != cudaSuccess) return fail(WAVE_ERR_CUDA, "cudaMemsetAsync(work counter): %s", cudaGetErrorString(e));
   rc = D == 128 ? launch<128>(prm, grid, s) : launch<64>(prm, grid, s);
@@ -977,8 +1007,9 @@ extern "C" int wave_round_attn_split(wave_kv* kv, const wave_node* active, int32
 // GPU that loads the library, until the process exits. Nothing is allocated
 // per call. Host code must not hand the array's name to a kernel (on the host
 // it is only a stand-in, not a device address); its device address is looked
-// up once per device with cudaGetSymbolAddress on the first call made with
-// that device current, and cached.
+// up with cudaGetSymbolAddress on the first call made with that device current
+// (again after a device reset, which gives the device a new context), and
+// cached.
 namespace wavei {
 namespace {
 constexpr int kStaticScratchWords = 64;    // 256 bytes per device
@@ -987,6 +1018,25 @@ constexpr int kMaxDevices = 64;
 static_assert(kStaticScratchNeeded <= kStaticScratchWords, "static scratch too small");
 std::mutex g_scratch_mu;
 int32_t* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};  // the context each address was looked up in
+
+// The calling thread's current context, from the driver (reached through the
+// runtime's entry-point query; null if unavailable).
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(f);
+  });
+  CUcontext ctx = nullptr;
+  if (fn) fn(&ctx);
+  return ctx;
+}
 }  // namespace
 }  // namespace wavei
 
@@ -1008,16 +1058,20 @@ extern "C" int wave_round_attn_static_scratch(wave_kv* kv, const wave_node* acti
   // The scratch need does not grow with the round (one counter), so the only
   // size limits are those wave_round_attn enforces: at most WAVE_MAX_NODES
   // nodes and WAVE_MAX_PAGES_PER_ROUND key pages (WAVE_ERR_CAPACITY beyond).
+  // Looked up once per device and context: a device reset makes a new
+  // context, in which the array lives at a new address.
   int32_t* scratch = nullptr;
   {
+    const CUcontext ctx = current_context();
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
       void* ptr = nullptr;
       e = cudaGetSymbolAddress(&ptr, g_round_attn_scratch);
       if (e != cudaSuccess || !ptr)
         return fail(WAVE_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s",
                     cudaGetErrorString(e));
       g_scratch_addr[dev] = static_cast<int32_t*>(ptr);
+      g_scratch_ctx[dev] = ctx;
     }
     scratch = g_scratch_addr[dev];
   }

@@ -450,6 +450,8 @@ extern "C" int wave_qkv_append_round(wave_kv* kv, const wave_node* nodes, int32_
     return fail(WAVE_ERR_ARG, "need 1..%d nodes, got %d", WAVE_MAX_NODES, n_nodes);
   if (!qkv_wide_supported(kv))
     return fail(WAVE_ERR_UNSUPPORTED, "the round projection needs head_dim 128 and 3 * heads even");
+  if (kv->fp8) return fail(WAVE_ERR_UNSUPPORTED, "the fused projection writes bf16 pages; "
+                           "append to an FP8 pool with wave_kv_append_batch");
   if (!X || !W || !Q || !aligned16(X) || !aligned16(W) || !aligned16(Q))
     return fail(WAVE_ERR_ARG, "X, W and Q must be non-NULL and 16-byte aligned");
   if (dim < 64 || dim % 64 != 0 || dim > (1 << 16))

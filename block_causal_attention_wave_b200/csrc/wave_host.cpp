@@ -123,12 +123,18 @@ int wave_kv_create(const wave_kv_config* cfg, wave_kv** out) {
     return fail(WAVE_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are built", cfg->head_dim);
   if (cfg->pool && (reinterpret_cast<uintptr_t>(cfg->pool) & 255))
     return fail(WAVE_ERR_ARG, "pool must be 256-byte aligned");
+  if (cfg->kv_format != WAVE_KV_BF16 && cfg->kv_format != WAVE_KV_FP8_E4M3)
+    return fail(WAVE_ERR_ARG, "unknown kv_format %d", cfg->kv_format);
   wave_kv* kv = new wave_kv();
   kv->cfg = *cfg;
-  kv->page_bytes = 2LL * cfg->heads * kPageTokens * cfg->head_dim * 2;
+  kv->fp8 = cfg->kv_format == WAVE_KV_FP8_E4M3;
+  kv->page_bytes = 2LL * cfg->heads * kPageTokens * cfg->head_dim * (kv->fp8 ? 1 : 2);
   kv->data_offset = kHeaderBytes;
-  int64_t avail = (int64_t)cfg->pool_bytes - kv->data_offset;
-  int64_t pages = avail > 0 ? avail / kv->page_bytes : 0;
+  // An FP8 page also needs its 2 H float32 scales (table after the pages,
+  // 256-byte aligned).
+  const int64_t per_page = kv->page_bytes + (kv->fp8 ? 2LL * cfg->heads * 4 : 0);
+  int64_t avail = (int64_t)cfg->pool_bytes - kv->data_offset - (kv->fp8 ? 256 : 0);
+  int64_t pages = avail > 0 ? avail / per_page : 0;
   // Row coordinates of the pool's tensor map are int32: pages * 2H * 128 < 2^31.
   int64_t max_by_coord = ((int64_t)1 << 31) / (2LL * cfg->heads * kPageTokens) - 1;
   pages = std::min<int64_t>(pages, std::min<int64_t>(max_by_coord, (1 << 25) - 1));
@@ -139,6 +145,7 @@ int wave_kv_create(const wave_kv_config* cfg, wave_kv** out) {
                                                                   cfg->head_dim * 2));
   }
   kv->max_pages = (int32_t)pages;
+  if (kv->fp8) kv->scale_offset = (kv->data_offset + pages * kv->page_bytes + 255) / 256 * 256;
   for (int32_t p = 0; p < kv->max_pages; ++p) kv->free_pages.insert(kv->free_pages.end(), p);
   kv->on_device = cfg->pool != nullptr;
   if (kv->on_device) {
@@ -215,6 +222,14 @@ int wave_kv_release(wave_kv* kv, int32_t chunk, int32_t level) {
     return fail(WAVE_ERR_MISSING_KV, "(%d, %d) is not cached", chunk, level);
   for (int32_t p : it->second.pages) kv->free_pages.insert(p);
   kv->entries.erase(it);
+  return WAVE_OK;
+}
+
+int wave_kv_scale_offset(const wave_kv* kv, int64_t* offset) {
+  clear_error();
+  if (!kv || !offset) return fail(WAVE_ERR_ARG, "NULL argument");
+  if (!kv->fp8) return fail(WAVE_ERR_ARG, "not an FP8 pool");
+  *offset = kv->scale_offset;
   return WAVE_OK;
 }
 

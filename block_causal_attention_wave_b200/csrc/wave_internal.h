@@ -29,6 +29,8 @@ struct wave_kv {
   int device = -1;
   int num_sms = 0;
   uint64_t wait_ns = 0;     // bound on one device wait; 0 = the default (2 s)
+  bool fp8 = false;         // pages hold E4M3 codes with per-(page, head) scales
+  int64_t scale_offset = 0; // FP8: byte offset of the scale table in the pool
   alignas(64) CUtensorMap tm_kv;  // rows of d bf16 over every page's K and V
 };
 
@@ -73,8 +75,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 bool qkv_wide_supported(const wave_kv* kv);
 int qkv_wide_launch(wave_kv* kv, int32_t n, const wave_node* nodes, int32_t T, const void* X,
                     int32_t dim, const void* W, const wave_rope* rope, void* Q, void* stream);
+// bf16 bytes of one page (the layout the attention kernel reads).
+inline int64_t bf16_page_bytes(const wave_kv* kv) {
+  return 2LL * kv->cfg.heads * WAVE_PAGE_TOKENS * kv->cfg.head_dim * 2;
+}
+// FP8 pools: expand `n` pages (ids in `pages`) into bf16 pages at `staging`
+// (slot i = pages[i]), the read-back bf16(code * scale), one launch.
+int launch_fp8_expand(wave_kv* kv, int32_t n, const int32_t* pages, void* staging, void* stream);
 // One kernel launch copying the K/V of n entries (already allocated) into
-// their pages.
+// their pages (quantising them for an FP8 pool).
 int launch_append(wave_kv* kv, int32_t n, const wave_entry* const* entries,
                   const void* const* K, const void* const* V, void* stream);
 

@@ -266,6 +266,8 @@ extern "C" int wave_qkv_append(wave_kv* kv, int32_t chunk, int32_t level, const 
   if (!kv) return fail(WAVE_ERR_ARG, "NULL handle");
   if (!kv->on_device) return fail(WAVE_ERR_ARG, "host-only handle (pool == NULL) cannot append");
   if (int rc = check_current_device(kv)) return rc;
+  if (kv->fp8) return fail(WAVE_ERR_UNSUPPORTED, "the fused projection writes bf16 pages; "
+                           "append to an FP8 pool with wave_kv_append");
   if (!X || !W || !Q ||
       ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(Q)) & 15))
     return fail(WAVE_ERR_ARG, "X, W and Q must be non-NULL and 16-byte aligned");

@@ -83,14 +83,28 @@ typedef struct {
                                NULL for a host-only handle (tables, no kernels)   */
   uint64_t pool_bytes;      /* size of pool (for a host-only handle: the size the
                                page count is derived from)                       */
+  int32_t kv_format;        /* WAVE_KV_BF16 (0) or WAVE_KV_FP8_E4M3              */
 } wave_kv_config;
+
+/* Page formats. BF16: K and V as bf16. FP8_E4M3: K and V as E4M3 codes (1
+ * sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448),
+ * each (page, head) tile of K and of V with one float32 scale: s = amax / 448
+ * over the tile's 128 token rows (1 if amax = 0), code = E4M3(x / s) with
+ * round to nearest even and saturation; the attention reads bf16(code * s).
+ * This halves the bytes of every cached entry -- the pages leave K/V cache
+ * growth open ([WS], limitations), and the same-level policy keeps K levels of
+ * history alive ([DS] Table 1). */
+#define WAVE_KV_BF16     0
+#define WAVE_KV_FP8_E4M3 1
 
 /* Create a paged (chunk, level) K/V cache over cfg->pool ([WF] history cache,
  * [WS] "K/V cache"). The pool holds a 4096-byte header (the device status
  * word at byte 0, the attention kernel's work-queue counter at byte 128, the
  * last attention launch's clock words at bytes 256..271) and
- * then pages of 2*H*128*d bf16 values: K as [H][128][d], then V as
- * [H][128][d]. Page p starts at pool + data_offset + p * page_bytes. With a
+ * then pages of 2*H*128*d values (bf16, or E4M3 codes for WAVE_KV_FP8_E4M3):
+ * K as [H][128][d], then V as [H][128][d]. Page p starts at pool +
+ * data_offset + p * page_bytes. FP8 pools hold after the last page (at
+ * wave_kv_scale_offset) the scales, float32 [max_pages][2 (K, V)][H]. With a
  * non-NULL pool this call clears the header synchronously and needs a CUDA
  * device with sm_100. *out receives the handle; destroy it with
  * wave_kv_destroy. Errors: ARG (bad sizes, misaligned pool, pool too small),
@@ -103,6 +117,10 @@ int wave_kv_destroy(wave_kv* kv);
 /* Report the pool layout: bytes per page, byte offset of page 0, page count. */
 int wave_kv_pool_layout(const wave_kv* kv, int64_t* page_bytes, int64_t* data_offset,
                         int32_t* max_pages);
+
+/* Byte offset (from the pool's start) of an FP8 pool's scale table,
+ * float32 [max_pages][2][H]. Errors: ARG (not an FP8 handle). */
+int wave_kv_scale_offset(const wave_kv* kv, int64_t* offset);
 
 /* Reserve pages for entry (chunk, level) holding ntokens tokens without
  * writing them: ceil(ntokens/128) pages, each the lowest free page id, taken
@@ -269,17 +287,22 @@ int wave_round_attn(wave_kv* kv, const wave_node* active, int32_t n_active, int3
  * softmax(Q K^T / sqrt(d)) V as wave_round_attn, up to rounding.
  * splits: >= 1 ranges per item (at most 32), or 0 = enough to give the GPU
  * about two waves of items (1 when the round already has a wave of them).
- * workspace: device buffer, 16-byte aligned, at least the bytes
+ * workspace: device buffer, 256-byte aligned, at least the bytes
  * wave_round_attn_split_workspace reports for the same arguments (none is
  * needed when no node is split); caller-owned, its contents are scratch.
+ * For an FP8 pool the workspace also holds, first, the round's distinct pages
+ * expanded to bf16 (one launch before the attention reads them), so an FP8
+ * pool needs a workspace even with splits = 1; wave_round_attn and
+ * wave_round_attn_static_scratch refuse FP8 pools (ARG).
  * Other arguments, layouts, limits and errors as wave_round_attn; ARG also
- * for a missing or too small workspace. */
+ * for a missing, misaligned (256 bytes) or too small workspace. */
 int wave_round_attn_split(wave_kv* kv, const wave_node* active, int32_t n_active, int32_t policy,
                           int32_t splits, const void* Q, void* O, void* workspace,
                           uint64_t workspace_bytes, void* stream);
 
 /* Workspace bytes wave_round_attn_split needs for these arguments (0 if no
- * node ends up split) and, in *splits_used (may be NULL), the ranges per item
+ * node ends up split and the pool is bf16) and, in *splits_used (may be
+ * NULL), the ranges per item
  * it will use (splits = 0 resolved). Host only. Errors: as wave_round_attn's
  * table checks (ARG, MISSING_KV, CAPACITY). */
 int wave_round_attn_split_workspace(wave_kv* kv, const wave_node* active, int32_t n_active,
@@ -300,7 +323,10 @@ int wave_round_attn_split_workspace(wave_kv* kv, const wave_node* active, int32_
  * wave_kv_status. It allocates nothing: no cudaMalloc/cudaFree, no library
  * allocator. The first call on a device, made with that device current (it
  * must be the pool's device), looks up the array's device address once and
- * caches it; make that first call before any stream capture. Each call zeroes
+ * caches it (per device and context: after a device reset, which gives the
+ * device a new context, the next call looks it up again); make that first
+ * call, and the first after a reset, before any stream capture. A reset also
+ * ends every handle made before it. Each call zeroes
  * the counter on `stream` before its launch. All calls on a device share the
  * one array: calls whose kernels overlap on the GPU (e.g. on two streams
  * without ordering) race on it and give undefined results. */

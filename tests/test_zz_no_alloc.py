@@ -7,9 +7,10 @@ wave_round_attn_static_scratch, which keeps the kernel's work-queue counter in
 a static device array inside the library instead of the pool header. This test
 runs it twice in a row through the C ABI and checks both outputs against
 wave_round_attn's on the same inputs, with the tolerance of the other parity
-tests (max-abs <= 1e-2, rel-L2 <= 5e-3). The second call only matches if the
-first left nothing behind that the second depends on (each call zeroes the
-counter before its launch).
+tests (max-abs <= 1e-2, rel-L2 <= 5e-3), and requires the bytes to equal
+wave_round_attn's exactly, since both run the same kernel and arithmetic. The
+second call only matches if the first left nothing behind that the second
+depends on (each call zeroes the counter before its launch).
 
 The file is named to be collected last, so a run that stops at the first
 failure has already run every other test.
@@ -53,5 +54,10 @@ def test_static_scratch_matches_wave_round_attn(cuda_lib, wl):
         o = torch.full_like(q, float("nan"))
         kv.round_attn_static_scratch(active, pol, q, o)
         kv.status()
+        # Same kernel, same arithmetic: only the counter's address differs, so
+        # the bytes must match exactly (a skipped or doubled work item would
+        # show here even where a tolerance would hide it).
+        assert not torch.isnan(o).any(), f"{wl.name} call {call + 1}: rows left unwritten"
+        assert torch.equal(o, o_ref), f"{wl.name} static-scratch call {call + 1}"
         assert_close(torch_to_f64(o), ref, f"{wl.name} static-scratch call {call + 1}")
     del keep
