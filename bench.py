@@ -105,6 +105,28 @@ def _measured_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
+def _source_hash(names):
+    import hashlib
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "block_causal_attention_wave_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _measured_append_traffic():
+    """DRAM bytes of the batched append launch from the committed ncu record, if
+    it was taken on the current append source (else None)."""
+    path = os.path.join(ROOT, "profiles", "kv_append_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != _source_hash(["wave_device.cu"]):
+        return None
+    return {k: rec.get(k) for k in ("dram_read_bytes", "dram_write_bytes", "duration_ns")}
+
+
 def _measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -521,7 +543,10 @@ def run_gpu(args):
                    "achieved_gbs": round(append_bytes / (append_ms * 1e-3) / 1e9, 1),
                    "peak_gbs": peaks["hbm_gbs"],
                    "frac": round(append_bytes / (append_ms * 1e-3) / 1e9 /
-                                 peaks["hbm_gbs"], 4)},
+                                 peaks["hbm_gbs"], 4),
+                   "ncu": _measured_append_traffic(),
+                   "ncu_note": "DRAM bytes of one batched append launch (ncu): writes that are "
+                               "still in L2 when the kernel ends reach DRAM later"},
         "gpu_launches": K * 2,
         "updates_only": updates,
         "projection": proj,

@@ -782,16 +782,25 @@ namespace {
 // int32 that this call sets to zero on `stream` before the launch).
 // Key ranges per (node, head, pair) for a call: `splits` >= 1 as asked; 0 =
 // none when the round already has a wave of items for the SMs (the dynamic
-// longest-first queue balances those), else enough for about two waves; at
-// most the node's pages and kMaxSplits.
+// longest-first queue balances those), else the fewest ranges whose items
+// fill their last wave of SMs to at least 90 % (the best fill found if none
+// does); at most the node's pages and kMaxSplits.
 constexpr int kMaxSplits = 32;
 int choose_splits(const wave_kv* kv, int32_t n_active, int32_t splits) {
   if (splits > 0) return std::min(splits, kMaxSplits);
   const int T = kv->cfg.tokens_per_chunk, H = kv->cfg.heads;
   const int64_t items = (int64_t)n_active * H * (((T + 127) / 128 + 1) / 2);
   if (items >= kv->num_sms) return 1;
-  const int64_t want = 2LL * kv->num_sms;
-  return (int)std::min<int64_t>(kMaxSplits, (want + items - 1) / items);
+  int best = 1;
+  double best_fill = 0.0;
+  for (int s = 2; s <= kMaxSplits; ++s) {
+    const int64_t n = items * s;
+    const int64_t waves = (n + kv->num_sms - 1) / kv->num_sms;
+    const double fill = (double)n / (double)(waves * kv->num_sms);
+    if (fill >= 0.9) return s;
+    if (fill > best_fill) best_fill = fill, best = s;
+  }
+  return best;
 }
 
 // Bytes of workspace a split call needs: per work item and query tile, 128
