@@ -13,7 +13,9 @@
 //
 // How (one kernel, B200 design): C = A B^T with A [M][K] and B [N][K] both
 // K-major bf16, tiles of 128 rows x 256 columns, one persistent CTA per SM
-// walking its tiles (consecutive tiles share a B tile, so it stays in L2).
+// walking its tiles. Tiles run row-tile-major: concurrent CTAs share A row
+// tiles, and B (the weights, at most a few tens of MB) stays in L2, so A -- the
+// activations, up to hundreds of MB -- comes from DRAM once.
 // 192 threads:
 //   warp 0 lane 0  TMA producer: 64-column slices of the A and B tiles
 //                  (128-byte swizzle) into a 4-stage shared-memory ring that
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * C::kBars + 4);
   const Ctl ctl{abort_flag, p.status, p.wait_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = p.k_slices, n_tiles = p.n_tiles, n_m = p.n_mtiles;
+  const int nk = p.k_slices, n_tiles = p.n_tiles, n_n = p.n_ntiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t g = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int nt = t / n_m, mt = t - nt * n_m;
+        const int mt = t / n_n, nt = t - mt * n_n;
         const int32_t row0 = (int32_t)a_row0(p, mt);
         for (int k = 0; k < nk; ++k, ++g) {
           const uint32_t s = g % S;
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __all_sync(0xffffffffu, wait_bar(bar(C::kAccFull + acc), (i >> 1) & 1, ctl, 0x304));
       if (!ok) break;
       tc_fence_after();
-      const int nt = t / n_m, mt = t - nt * n_m;
+      const int mt = t / n_n, nt = t - mt * n_n;
       if (p.mode == MODE_LINEAR) {
         const int64_t r = (int64_t)mt * 128 + row;
         const bool in = r < p.M;
