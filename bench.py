@@ -391,24 +391,26 @@ def run_gpu(args):
 
     # ---- fused QKV projection + K/V append of the round's nodes (the step
     # that produces the K/V the round appends), random Wan2.1-shaped weights:
-    # X [T][C] per node, W [3 H d][C]. A sleep kernel keeps the GPU busy while
-    # the host enqueues, so the events see only the launches.
+    # X [5 T][C] for the round's nodes, W [3 H d][C]; ONE launch for the round
+    # (wave_qkv_append_round, no rotary here: the block line below has it). A
+    # sleep kernel keeps the GPU busy while the host enqueues, so the events see
+    # only the launches.
     proj = None
-    if wl.head_dim in (64, 128) and spec.key == DEFAULT_WORKLOAD:
-        dim = 1536  # Wan2.1-1.3B hidden size
-        xs = [_bits_to_dev(wi.hidden_states(n[0], n[1], wl.tokens, dim)) for n in active]
+    if wl.head_dim == 128 and (3 * wl.heads) % 2 == 0 and spec.key == DEFAULT_WORKLOAD:
+        dim = wi.WAN21_DIM
+        X = torch.cat([_bits_to_dev(wi.hidden_states(n[0], n[1], wl.tokens, dim)) for n in active])
         wqkv = _bits_to_dev(wi.qkv_weight(wl.heads, wl.head_dim, dim))
-        qp = torch.empty(wl.tokens, wl.heads, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+        qp = torch.empty(len(active) * wl.tokens, wl.heads, wl.head_dim, dtype=torch.bfloat16,
+                         device="cuda")
 
         def proj_round():
-            for n, x in zip(active, xs):
-                kv.qkv_append(n[0], n[1], x, wqkv, qp, stream)
+            kv.qkv_append_round(active, X, wqkv, qp, stream=stream)
             for n in active:
                 kv.release(*n)
 
         proj_round()
         torch.cuda.synchronize()
-        reps = 5
+        reps = 10
         pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda._sleep(int(3e6))
         pa.record(stream)
@@ -417,12 +419,11 @@ def run_gpu(args):
         pb.record(stream)
         torch.cuda.synchronize()
         kv.status(stream)
-        p_ms = pa.elapsed_time(pb) / (reps * len(active))
-        p_flops = 2 * wl.tokens * 3 * wl.heads * wl.head_dim * dim
-        wide = wl.head_dim == 128 and (3 * wl.heads) % 2 == 0
-        proj = {"kernel": "qkv_append_wide_kernel" if wide else "qkv_append_kernel<%d>" % wl.head_dim,
-                "what": "Q,K,V = X W^T per node, K/V written "
-                "into the node's new pages in the epilogue", "dim": dim,
+        p_ms = pa.elapsed_time(pb) / reps
+        p_flops = 2 * len(active) * wl.tokens * 3 * wl.heads * wl.head_dim * dim
+        proj = {"kernel": "gemm_wide_kernel (QKV epilogue)",
+                "what": "Q,K,V = X W^T for the round's 5 nodes in one launch, K/V written "
+                "into each node's new pages in the epilogue", "dim": dim,
                 "flops_per_launch": p_flops, "avg_launch_ms": round(p_ms, 4),
                 "achieved": round(p_flops / (p_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "frac": round(p_flops / (p_ms * 1e-3) / 1e12 / _measured_peaks()[0]["bf16_tflops"],
