@@ -58,8 +58,23 @@ int main(void) {
   rc = wave_gather_table(kv, act, 1, WAVE_POLICY_SAME, rows, roffs, 8, &n_rows);
   CHECK(rc == WAVE_ERR_MISSING_KV, "same-level needs E(0, 1): MISSING_KV");
 
+  int32_t own[4], n_own = 0;
+  CHECK(wave_kv_entry_pages(kv, 1, 1, own, 4, &n_own) == WAVE_OK && n_own == 2 && own[0] == 2 &&
+            own[1] == 3, "entry pages of (1, 1) are 2, 3");
+  CHECK(wave_kv_set_wait_limit(kv, 5000) == WAVE_OK, "wait limit set");
   CHECK(wave_kv_release(kv, 0, 0) == WAVE_OK, "release (0, 0)");
   CHECK(wave_kv_free_pages(kv, &free_pages) == WAVE_OK && free_pages == 6, "6 free pages");
+
+  /* Wave Parallelism, progressive, B = 3, K = 2 on 3 ranks: round 2 runs
+   * (0, 0), (1, 1), (2, 2); E(0, 0) goes from rank 0 to ranks 1 and 2. */
+  wave_transfer tr[8];
+  int32_t n_tr = 0;
+  rc = wave_wp_transfers(3, 2, WAVE_POLICY_PROGRESSIVE, 0, 3, 2, tr, 8, &n_tr);
+  CHECK(rc == WAVE_OK && n_tr >= 2 && tr[0].chunk == 0 && tr[0].level == 0 && tr[0].src == 0,
+        "round 2 pushes E(0, 0) from rank 0");
+  int all_one_way = 1;
+  for (int32_t i = 0; i < n_tr; ++i) all_one_way &= tr[i].dst > tr[i].src;
+  CHECK(all_one_way, "progressive pushes go from a cleaner to a noisier rank");
   CHECK(strlen(wave_strerror(WAVE_ERR_NO_PAGES)) > 0, "strerror names codes");
   CHECK(wave_kv_destroy(kv) == WAVE_OK, "destroy");
   return 0;

@@ -184,3 +184,37 @@ def test_fp8_pool_refuses_what_needs_bf16_pages(cuda_lib):
         kv.qkv_append(1, 1, x, w, torch.empty((128, 2, 128), dtype=torch.bfloat16, device="cuda"))
     assert kv.split_workspace([(0, 1)], "progressive", 1)[0] > 0
     del keep
+
+
+def test_fp8_pool_with_split_key_ranges(cuda_lib):
+    """FP8 pages and split key ranges together: the workspace holds the bf16
+    staging pages first and the ranges' partial results after them."""
+    wave = cuda_lib
+    wl = wi.Workload("fp8-split", chunks=5, levels=2, heads=2, head_dim=128, tokens=300,
+                     prefix=77)
+    pol = "progressive"
+    inp = Inputs(wl)
+    orc = _Oracle(inp)
+    kv, _ = _fp8_cache(wave, wl, 80)
+    active = max(osched.schedule(wl.chunks, wl.levels, pol, wl.window),
+                 key=lambda r: (len(r), r[-1][0]))
+    ents = set()
+    for n in active:
+        ents.update(ocache.key_entries(n, pol, wl.window, True))
+    keep = [_append(kv, inp, e) for e in sorted(ents)]
+    import torch
+    q = queries(inp, active)
+    o = torch.full_like(q, float("nan"))
+    nbytes, used = kv.split_workspace(active, pol, 3)
+    assert used == 3 and nbytes > kv.split_workspace(active, pol, 1)[0]
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    kv.round_attn_split(active, pol, q, o, ws, 3)
+    kv.status()
+    needed = set(e for n in active for e in ocache.key_entries(n, pol, wl.window, True)
+                 if e != ocache.PREFIX)
+    ref = oatt.round_attention(active, pol, wl.window, {n: inp.f64("q", *n) for n in active},
+                               {e: orc.readback(e) for e in needed}, orc.readback((-1, 0)))
+    got = torch_to_f64(o).reshape(len(active), wl.tokens, wl.heads, wl.head_dim)
+    for i, n in enumerate(active):
+        assert_close(got[i], ref[n], f"fp8 + 3 ranges, node {n}")
+    del keep

@@ -162,3 +162,40 @@ def test_random_rollouts_match_oracle_bit_exact(lib):
         got = _library_rollout(wl, pol, max_pages)
         want = ocache.rollout_tables(B, K, pol, W, T, prefix, max_pages)
         assert got == [(a, t) for a, t in want], (B, K, W, T, prefix, pol)
+
+
+def test_host_only_handle_refuses_device_calls_of_the_block_and_split(lib):
+    """Calls that launch kernels refuse a host-only handle before any work."""
+    import ctypes
+    import block_causal_attention_wave_b200 as wave
+    from block_causal_attention_wave_b200 import _binding as b
+    kv = wave.KVCache(2, 128, 256, 2, pool=None, pool_bytes=4096 + 16 * wave.KVCache.page_bytes(2, 128))
+    node = (b.Node * 1)(b.Node(0, 1))
+    nbytes, used = ctypes.c_uint64(), ctypes.c_int32()
+    assert lib.wave_round_attn_split_workspace(kv.h, node, 1, 2, 0, ctypes.byref(nbytes),
+                                               ctypes.byref(used)) == b.ERR_ARG
+    assert lib.wave_round_attn_split(kv.h, node, 1, 2, 0, None, None, None, 0, None) == b.ERR_ARG
+    assert lib.wave_qkv_append_round(kv.h, node, 1, None, 128, None, None, None, None) == b.ERR_ARG
+    assert lib.wave_linear(kv.h, None, 128, 128, None, 256, None, 0, None, None) == b.ERR_ARG
+    off = ctypes.c_int64()
+    assert lib.wave_kv_scale_offset(kv.h, ctypes.byref(off)) == b.ERR_ARG  # not an FP8 pool
+    assert lib.wave_kv_set_wait_limit(kv.h, 1000) == b.OK
+    assert kv.free_pages() == 16  # nothing was taken
+
+
+def test_fp8_host_only_layout(lib):
+    """An FP8 pool's pages hold one-byte codes, and its scale table sits after
+    the last page, 256-byte aligned, with 2 H float32 per page."""
+    import block_causal_attention_wave_b200 as wave
+    H, d = 3, 128
+    pb8 = wave.KVCache.page_bytes(H, d, wave.KV_FP8_E4M3)
+    assert pb8 == 2 * H * 128 * d
+    pool_bytes = 4096 + 256 + 10 * (pb8 + 2 * H * 4)
+    kv = wave.KVCache(H, d, 300, 2, pool=None, pool_bytes=pool_bytes, kv_format=wave.KV_FP8_E4M3)
+    page_bytes, off, maxp = kv.layout()
+    assert page_bytes == pb8 and maxp == 10
+    soff = kv.scale_offset()
+    assert soff % 256 == 0 and soff >= off + maxp * pb8
+    assert soff + maxp * 2 * H * 4 <= pool_bytes
+    kv.alloc(0, 1)
+    assert kv.entry_pages(0, 1) == [0, 1, 2]
