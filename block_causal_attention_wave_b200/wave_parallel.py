@@ -56,16 +56,30 @@ class WaveParallel:
         incoming = sorted({e for e, _, dst in pushes if dst == self.rank})
         for e in incoming:
             self.kv.alloc(*e)
-        reqs = []
+        # NCCL moves device pages directly; a backend without device support
+        # (gloo) gets host copies of them.
+        staged = self.pool.is_cuda and dist.get_backend(self.group) != "nccl"
+        reqs, landing = [], []
+        if staged:
+            import torch
+            torch.cuda.current_stream().synchronize()  # the appends wrote the pages
         for e, src, dst in pushes:  # the same order on every rank
             if src == self.rank:
                 for p in self.kv.entry_pages(*e):
-                    reqs.append(dist.isend(self._page(p), dst, group=self.group))
+                    buf = self._page(p).cpu() if staged else self._page(p)
+                    reqs.append((dist.isend(buf, dst, group=self.group), buf))
             elif dst == self.rank:
                 for p in self.kv.entry_pages(*e):
-                    reqs.append(dist.irecv(self._page(p), src, group=self.group))
-        for r in reqs:
+                    if staged:
+                        buf = self._page(p).new_empty(self._page(p).shape, device="cpu")
+                        landing.append((p, buf))
+                    else:
+                        buf = self._page(p)
+                    reqs.append((dist.irecv(buf, src, group=self.group), buf))
+        for r, _ in reqs:
             r.wait()
+        for p, buf in landing:
+            self._page(p).copy_(buf)
         return incoming
 
     def release(self, t):
