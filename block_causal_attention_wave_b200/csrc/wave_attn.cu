@@ -31,8 +31,9 @@
 //            stale max is kept, exact after the final division as P <= 2^8
 //            stays inside fp32/bf16. Epilogue: O / l, bf16, stored straight
 //            from registers (only rows that belong to the node).
-// Every wait is bounded (2 s); on timeout the kernel records a status word,
-// every role stops, and TMEM is freed before exit.
+// Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
+// the kernel records a status word, every role stops, and TMEM is freed
+// before exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -58,8 +59,9 @@ namespace wavei {
 namespace {
 
 constexpr int kThreads = 384;  // warp 0 TMA, warps 1 and 3 MMA, warps 4..11 softmax (2 groups)
-// Register split after start-up (setmaxnreg): warps 0..3 (TMA, MMA, two idle;
-// one per SM sub-partition) drop to kRegsLow, the two softmax warpgroups (two
+// Register split after start-up (setmaxnreg): warps 0..3 (the TMA producer,
+// the two MMA issuers and one idle warp; one per SM sub-partition) drop to
+// kRegsLow, the two softmax warpgroups (two
 // warps per sub-partition) rise to kRegsHigh, so each softmax thread can hold
 // a full 128-column S row without spilling. Per sub-partition
 // kRegsLow + 2 kRegsHigh <= 504 registers per lane, i.e. at most what the
