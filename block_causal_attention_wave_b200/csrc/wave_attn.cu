@@ -22,7 +22,10 @@
 //            Pipe order per page t: S_0(t), PV_0(t-1), S_1(t), PV_1(t-1): the
 //            S buffer is reloaded while the P.V behind it runs, and a tile's
 //            P(t) is needed only after the next page's S. Two issuing threads
-//            keep the tensor pipe's short queue fed while either one waits.
+//            keep the tensor pipe's short queue fed while either one waits;
+//            they do nothing but wait for S_FREE / P_FULL, issue and commit
+//            (a tcgen05.mma call returns only about when the pipe takes it,
+//            so every other step on these threads delays the pipe).
 //   warps 4-11  softmax, one warpgroup per query tile, one row per thread:
 //            tcgen05.ld of the S row (then S is handed back), padding keys of
 //            a partial page masked, max in the log2 domain, exp2, bf16 P
@@ -30,7 +33,12 @@
 //            running max grows by more than 8 (log2 units); otherwise the
 //            stale max is kept, exact after the final division as P <= 2^8
 //            stays inside fp32/bf16. Epilogue: O / l, bf16, stored straight
-//            from registers (only rows that belong to the node).
+//            from registers (only rows that belong to the node). The softmax
+//            warpgroups also take ring work off the issuers: they check that
+//            the next S's K page and their own P.V's V page have landed before
+//            handing the S buffer / P_w over, and give each K slot back once
+//            they see the page's last S done (V slots go back by a commit
+//            behind each P.V).
 // Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
 // the kernel records a status word, every role stops, and TMEM is freed
 // before exit.
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_DRAIN + 1), 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(BR::RING_FULL + s), 1);
-      mbar_init(bar(BR::RING_EMPTY + s), 2);  // one commit from each MMA thread
+      mbar_init(bar(BR::RING_EMPTY + s), 2);  // K: one arrival of 2; V: a commit per tile
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -413,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!accumulate && itw > 0 &&
               !wait_bar(bar(B_O_EMPTY + mw), (itw - 1) & 1, ctl, 0x114 + mw))
             return false;
-          if (!ring_wait(2 * t + 1, 0x116 + mw)) return false;
+          // P_FULL implies V(t) has landed: the softmax checked it first.
           tc_fence_after();
           const uint32_t vaddr = slot_addr(2 * t + 1);
           mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * mw, tmem + C::kColP + 64 * mw,
@@ -422,11 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++pv;
           return true;
         };
-        // A ring slot is released by one commit from each MMA thread; with a
-        // single query tile, thread 0 gives both.
-        auto release = [&](uint32_t r, int nq) {
-          tc_commit(bar(BR::RING_EMPTY + r % S));
-          if (nq == 1) tc_commit(bar(BR::RING_EMPTY + r % S));
+        // V(t) goes back to the producer by one commit behind each tile's P.V
+        // (two from thread 0 with a single tile); K(t) by the softmax that
+        // sees the page's last S done.
+        auto release_v = [&](uint32_t t, int nq) {
+          tc_commit(bar(BR::RING_EMPTY + (2 * t + 1) % S));
+          if (nq == 1) tc_commit(bar(BR::RING_EMPTY + (2 * t + 1) % S));
         };
         // Pipe order per page t: S_0(t), PV_0(t-1) from thread 0 and S_1(t),
         // PV_1(t-1) from thread 1. A tile's P(t) is consumed after S of page
@@ -448,22 +457,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_bar(bar(B_Q_FULL), qit & 1, ctl, 0x110)) { ok = false; break; }
           for (int j = 0; j < n && ok; ++j, ++g) {
             if (mw == 1) take_s(0);  // thread 0's S_0(t) went first
-            // Thread 1's S follows S_0(t), whose S_FREE implies K(t) was in.
-            if (mw == 0 && !ring_wait(2 * g, 0x111)) { ok = false; break; }
+            // K(t) has landed: for an item's first page this thread checks;
+            // later, the S_FREE it waits for implies it (thread 1's S follows
+            // S_0(t); the softmax that frees the buffer for S_0(t) checked K(t)).
+            if (mw == 0 && j == 0 && !ring_wait(2 * g, 0x111)) { ok = false; break; }
             if (!issue_s(g)) { ok = false; break; }
             if (mw == nq - 1 && j == n - 1) tc_commit(bar(B_Q_EMPTY));  // the item's last S
-            release(2 * g, nq);  // K(t): this thread's S done
             if (mw == 0 && nq == 2) take_s(1);  // thread 1's S_1(t) follows
             if (j > 0) {
               if (!issue_pv(g - 1, j > 1)) { ok = false; break; }
-              release(2 * (g - 1) + 1, nq);  // V(t-1): this thread's P.V done
+              release_v(g - 1, nq);
             }
           }
           if (!ok) break;
           // The item's last page: this tile's P.V, then its O is complete.
           if (!issue_pv(g - 1, n > 1)) { ok = false; break; }
           tc_commit(bar(B_O_FULL + mw));
-          release(2 * (g - 1) + 1, nq);
+          release_v(g - 1, nq);
           ++itw;
         }
         // Wait (bounded) until every MMA issued by this thread has finished.
@@ -483,8 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = trow + C::kColO + 128 * wq;
     const float sl2 = p.scale_log2;
     // g: S tiles loaded, pw: P_w written (each one read by a P.V that commits
-    // P_FREE_w), it: items finished by this warpgroup.
-    uint32_t g = 0, pw = 0, it = 0;
+    // P_FREE_w), it: items finished by this warpgroup, gp: pages of every
+    // item so far, both tiles' (the ring holds K(gp) at 2 gp, V(gp) at 2 gp + 1).
+    uint32_t g = 0, pw = 0, it = 0, gp = 0;
+    // One thread per warpgroup checks that a ring slot has landed before the
+    // S buffer or P_w is handed to an MMA that reads it, and gives a K slot
+    // back (both of its expected arrivals) once the page's S MMAs are done.
+    const bool lead = quarter == 0 && lane == 0;
+    auto ring_landed = [&](uint32_t r, int code) -> bool {
+      return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
+    };
     for (uint32_t k = 0;; ++k) {
       Item w;
       bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, w));
@@ -492,13 +510,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
       if (w.id >= p.n_items) break;
-      if (wq == 1 && !w.two) continue;  // the pair's second tile lies past the node
+      if (wq == 1 && !w.two) {  // the pair's second tile lies past the node
+        gp += w.n_pages;
+        continue;
+      }
       const AttnNode& nd = p.nodes[w.node];
+      // This warpgroup loads each page's last S (so K(t) is free once it
+      // sees S_FULL) unless the pair's second tile follows.
+      const bool last_s = wq == 1 || !w.two;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int t = 0; t < w.n_pages; ++t, ++g) {
-        ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
+      for (int t = 0; t < w.n_pages; ++t, ++g, ++gp) {
+        // V(t) must be in before P_FULL hands P_w to the P.V; if this
+        // warpgroup's S_FREE lets S_0(t+1) go, K(t+1) must be in too.
+        bool in = true;
+        if (lead) {
+          in = ring_landed(2 * gp + 1, 0x128 + wq);
+          if (in && last_s && t + 1 < w.n_pages) in = ring_landed(2 * gp + 2, 0x128 + wq);
+        }
+        ok = __all_sync(0xffffffffu, in && wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
         tc_fence_after();
+        if (lead && last_s)  // both S MMAs of page t are done with K(t)
+          mbar_arrive_cnt(bar(BR::RING_EMPTY + (2 * gp) % S), 2);
         const int valid = (int)(p.pages[nd.page0 + w.page_begin + t] >> 25) + 1;
         // The whole S row in one TMEM round trip; then the S buffer goes back
         // to the MMA thread for the other tile's (or the next page's) S.
