@@ -33,12 +33,13 @@
 //            running max grows by more than 8 (log2 units); otherwise the
 //            stale max is kept, exact after the final division as P <= 2^8
 //            stays inside fp32/bf16. Epilogue: O / l, bf16, stored straight
-//            from registers (only rows that belong to the node). The softmax
-//            warpgroups also take ring work off the issuers: they check that
-//            the next S's K page and their own P.V's V page have landed before
-//            handing the S buffer / P_w over, and give each K slot back once
-//            they see the page's last S done (V slots go back by a commit
-//            behind each P.V).
+//            from registers (only rows that belong to the node). The warpgroup
+//            that sees a page's last S done gives its K slot back (V slots go
+//            back by a commit behind each P.V).
+//   warp 2   ring watcher: takes part in every S_FREE and P_FULL phase,
+//            arriving once the pages the MMAs behind it read have landed
+//            (K(t+1) for the S_FREE that lets S_0(t+1) go, V(t) for P_FULL),
+//            so neither the issuers nor the softmax wait on the ring.
 // Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
 // the kernel records a status word, every role stops, and TMEM is freed
 // before exit.
@@ -66,9 +67,9 @@ namespace wavei {
 
 namespace {
 
-constexpr int kThreads = 384;  // warp 0 TMA, warps 1 and 3 MMA, warps 4..11 softmax (2 groups)
+constexpr int kThreads = 384;  // warp 0 TMA, 1 and 3 MMA, 2 ring watcher, 4..11 softmax
 // Register split after start-up (setmaxnreg): warps 0..3 (the TMA producer,
-// the two MMA issuers and one idle warp; one per SM sub-partition) drop to
+// the two MMA issuers and the ring watcher; one per SM sub-partition) drop to
 // kRegsLow, the two softmax warpgroups (two
 // warps per sub-partition) rise to kRegsHigh, so each softmax thread can hold
 // a full 128-column S row without spilling. Per sub-partition
@@ -158,14 +159,14 @@ enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
   B_S_FULL,                  // 2: S = Q_w K^T computed into the S buffer
-  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (128 arrivals)
-  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (128 arrivals)
+  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (128 arrivals + the watcher)
+  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (128 arrivals + the watcher)
   B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
   B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
   B_DRAIN = B_O_EMPTY + 2,   // 2: every MMA of MMA thread w done (while stopping)
   B_ITEM_FULL = B_DRAIN + 2, // 2: next work item published by the producer
-  B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by the 2 MMA threads and 8 softmax warps
+  B_ITEM_EMPTY = B_ITEM_FULL + 2,  // 2: item read by 2 MMA threads, the watcher, 8 softmax warps
   B_RING_FULL = B_ITEM_EMPTY + 2,  // kSlots each from here
 };
 constexpr int kItemSlots = 2;
@@ -253,15 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_Q_EMPTY), 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(B_S_FULL + w), 1);
-      mbar_init(bar(B_S_FREE + w), 128);
-      mbar_init(bar(B_P_FULL + w), 128);
+      mbar_init(bar(B_S_FREE + w), 129);  // the warpgroup + the ring watcher
+      mbar_init(bar(B_P_FULL + w), 129);
       mbar_init(bar(B_P_FREE + w), 1);
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
     }
     for (int k = 0; k < kItemSlots; ++k) {
       mbar_init(bar(B_ITEM_FULL + k), 1);
-      mbar_init(bar(B_ITEM_EMPTY + k), 2 + 8);  // MMA threads + one lane per softmax warp
+      mbar_init(bar(B_ITEM_EMPTY + k), 3 + 8);  // MMA threads, watcher, one lane per softmax warp
     }
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_DRAIN + 1), 1);
@@ -355,6 +356,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q_last >= 0) drain_wait(bar(B_Q_FULL), (uint32_t)q_last);
           for (int s = 0; s < S; ++s)
             if (ring_last[s] >= 0) drain_wait(bar(BR::RING_FULL + s), (uint32_t)ring_last[s]);
+        }
+      }
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- ring watcher
+      // Takes part in every S_FREE and P_FULL phase, in order, arriving only
+      // once the ring slots the MMAs behind that phase read have landed:
+      // K(t+1) for an S_FREE that lets S_0(t+1) go, V(t) for a P_FULL. It
+      // arrives on a barrier's next phase only after the previous one
+      // completed, so it is never two phases ahead.
+      if (lane == 0) {
+        uint32_t g = 0, sf[2] = {0, 0}, pf[2] = {0, 0};
+        bool ok = true;
+        auto landed = [&](uint32_t r) -> bool {
+          return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, 0x12a);
+        };
+        auto next_phase = [&](int base, int w, uint32_t& n) -> bool {
+          if (n > 0 && !wait_bar(bar(base + w), (n - 1) & 1, ctl, 0x12b)) return false;
+          mbar_arrive(bar(base + w));
+          ++n;
+          return true;
+        };
+        for (uint32_t k = 0; ok; ++k) {
+          Item w;
+          if (!next_item(k, 0x12c, w)) break;
+          mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
+          if (w.id >= p.n_items) break;
+          const int nq = w.two ? 2 : 1;
+          for (int t = 0; ok && t < w.n_pages; ++t, ++g) {
+            for (int q = 0; ok && q < nq; ++q) {
+              // S_FREE_q(t): if it lets S_0(t+1) go, K(t+1) must be in.
+              if (q == nq - 1 && t + 1 < w.n_pages && !landed(2 * g + 2)) { ok = false; break; }
+              ok = next_phase(B_S_FREE, q, sf[q]);
+            }
+            if (!ok || !landed(2 * g + 1)) { ok = false; break; }
+            for (int q = 0; ok && q < nq; ++q) ok = next_phase(B_P_FULL, q, pf[q]);
+          }
         }
       }
     } else if (warp == 1 || warp == 3) {
@@ -497,13 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P_FREE_w), it: items finished by this warpgroup, gp: pages of every
     // item so far, both tiles' (the ring holds K(gp) at 2 gp, V(gp) at 2 gp + 1).
     uint32_t g = 0, pw = 0, it = 0, gp = 0;
-    // One thread per warpgroup checks that a ring slot has landed before the
-    // S buffer or P_w is handed to an MMA that reads it, and gives a K slot
-    // back (both of its expected arrivals) once the page's S MMAs are done.
+    // One thread per warpgroup gives a K slot back (both of its expected
+    // arrivals) once the page's S MMAs are done.
     const bool lead = quarter == 0 && lane == 0;
-    auto ring_landed = [&](uint32_t r, int code) -> bool {
-      return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, code);
-    };
     for (uint32_t k = 0;; ++k) {
       Item w;
       bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, w));
@@ -521,14 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool last_s = wq == 1 || !w.two;
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < w.n_pages; ++t, ++g, ++gp) {
-        // V(t) must be in before P_FULL hands P_w to the P.V; if this
-        // warpgroup's S_FREE lets S_0(t+1) go, K(t+1) must be in too.
-        bool in = true;
-        if (lead) {
-          in = ring_landed(2 * gp + 1, 0x128 + wq);
-          if (in && last_s && t + 1 < w.n_pages) in = ring_landed(2 * gp + 2, 0x128 + wq);
-        }
-        ok = __all_sync(0xffffffffu, in && wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
+        ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
         tc_fence_after();
         if (lead && last_s)  // both S MMAs of page t are done with K(t)
