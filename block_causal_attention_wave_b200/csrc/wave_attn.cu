@@ -33,13 +33,13 @@
 //            running max grows by more than 8 (log2 units); otherwise the
 //            stale max is kept, exact after the final division as P <= 2^8
 //            stays inside fp32/bf16. Epilogue: O / l, bf16, stored straight
-//            from registers (only rows that belong to the node). The warpgroup
-//            that sees a page's last S done gives its K slot back (V slots go
-//            back by a commit behind each P.V).
+//            from registers (only rows that belong to the node).
 //   warp 2   ring watcher: takes part in every S_FREE and P_FULL phase,
 //            arriving once the pages the MMAs behind it read have landed
 //            (K(t+1) for the S_FREE that lets S_0(t+1) go, V(t) for P_FULL),
-//            so neither the issuers nor the softmax wait on the ring.
+//            and gives each K slot back once the page's last S has been
+//            loaded (V slots go back by a commit behind each P.V), so neither
+//            the issuers nor the softmax do any ring work.
 // Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
 // the kernel records a status word, every role stops, and TMEM is freed
 // before exit.
@@ -159,8 +159,8 @@ enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
   B_S_FULL,                  // 2: S = Q_w K^T computed into the S buffer
-  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (128 arrivals + the watcher)
-  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (128 arrivals + the watcher)
+  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (4 warp arrivals + the watcher)
+  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (4 warp arrivals + the watcher)
   B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
   B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
@@ -254,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_Q_EMPTY), 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(B_S_FULL + w), 1);
-      mbar_init(bar(B_S_FREE + w), 129);  // the warpgroup + the ring watcher
-      mbar_init(bar(B_P_FULL + w), 129);
+      mbar_init(bar(B_S_FREE + w), 5);  // the warpgroup's 4 warps + the ring watcher
+      mbar_init(bar(B_P_FULL + w), 5);
       mbar_init(bar(B_P_FREE + w), 1);
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
@@ -364,7 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // once the ring slots the MMAs behind that phase read have landed:
       // K(t+1) for an S_FREE that lets S_0(t+1) go, V(t) for a P_FULL. It
       // arrives on a barrier's next phase only after the previous one
-      // completed, so it is never two phases ahead.
+      // completed, so it is never two phases ahead. Once page t's last S has
+      // been loaded (its S_FREE phase complete), both S MMAs are done with
+      // K(t) and the watcher gives that slot back (both expected arrivals).
       if (lane == 0) {
         uint32_t g = 0, sf[2] = {0, 0}, pf[2] = {0, 0};
         bool ok = true;
@@ -389,6 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (q == nq - 1 && t + 1 < w.n_pages && !landed(2 * g + 2)) { ok = false; break; }
               ok = next_phase(B_S_FREE, q, sf[q]);
             }
+            // Page t's last S was loaded once that S_FREE completes: K(t) goes back.
+            if (ok) ok = wait_bar(bar(B_S_FREE + nq - 1), (sf[nq - 1] - 1) & 1, ctl, 0x12d);
+            if (ok) mbar_arrive_cnt(bar(BR::RING_EMPTY + (2 * g) % S), 2);
             if (!ok || !landed(2 * g + 1)) { ok = false; break; }
             for (int q = 0; ok && q < nq; ++q) ok = next_phase(B_P_FULL, q, pf[q]);
           }
@@ -534,9 +539,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P_FREE_w), it: items finished by this warpgroup, gp: pages of every
     // item so far, both tiles' (the ring holds K(gp) at 2 gp, V(gp) at 2 gp + 1).
     uint32_t g = 0, pw = 0, it = 0, gp = 0;
-    // One thread per warpgroup gives a K slot back (both of its expected
-    // arrivals) once the page's S MMAs are done.
-    const bool lead = quarter == 0 && lane == 0;
     for (uint32_t k = 0;; ++k) {
       Item w;
       bool ok = __all_sync(0xffffffffu, next_item(k, 0x124 + wq, w));
@@ -549,16 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const AttnNode& nd = p.nodes[w.node];
-      // This warpgroup loads each page's last S (so K(t) is free once it
-      // sees S_FULL) unless the pair's second tile follows.
-      const bool last_s = wq == 1 || !w.two;
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < w.n_pages; ++t, ++g, ++gp) {
         ok = __all_sync(0xffffffffu, wait_bar(bar(B_S_FULL + wq), g & 1, ctl, 0x120 + wq));
         if (!ok) break;
         tc_fence_after();
-        if (lead && last_s)  // both S MMAs of page t are done with K(t)
-          mbar_arrive_cnt(bar(BR::RING_EMPTY + (2 * gp) % S), 2);
+
         const int valid = (int)(p.pages[nd.page0 + w.page_begin + t] >> 25) + 1;
         // The whole S row in one TMEM round trip; then the S buffer goes back
         // to the MMA thread for the other tile's (or the next page's) S.
@@ -568,7 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(bar(B_S_FREE + wq));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + wq));
         if (valid < 128) {  // partial last page of an entry: drop the padding keys
 #pragma unroll
           for (int i = 0; i < 128; ++i) sv[i] = i < valid ? sv[i] : -INFINITY;
@@ -663,7 +662,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run += (acc[0] + acc[1]) + (acc[2] + acc[3]);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + wq));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_P_FULL + wq));
         ++pw;
       }
       if (!ok) break;
