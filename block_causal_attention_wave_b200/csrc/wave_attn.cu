@@ -119,10 +119,10 @@ struct AttnParams {
 static_assert(sizeof(AttnParams) <= 32760, "kernel parameter space is 32 KB");
 
 // Softmax columns (of each 32) whose exp2 runs on the FMA pipe (polynomial)
-// instead of the special-function unit; even, 0..32. Four: in long runs under
-// the power cap, 4 and 0 took about 1.5 % fewer cycles per launch than 8.
+// instead of the special-function unit; even, 0..32. Two: measured against
+// 0, 4, 6 and 8, it took the fewest cycles per launch (8 about 4 % more).
 #ifndef WAVE_EMU_PER_CHUNK
-#define WAVE_EMU_PER_CHUNK 4
+#define WAVE_EMU_PER_CHUNK 2
 #endif
 constexpr int kEmuPerChunk = WAVE_EMU_PER_CHUNK;
 // 1: scale/shift of S and the row sum use packed fp32x2 FMA/ADD.
