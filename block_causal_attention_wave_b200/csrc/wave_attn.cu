@@ -40,6 +40,10 @@
 //            and gives each K slot back once the page's last S has been
 //            loaded (V slots go back by a commit behind each P.V), so neither
 //            the issuers nor the softmax do any ring work.
+// A node's last pair of query tiles may hold one tile. The S tiles of such a
+// single-tile item signal a third S_FREE barrier: thread 1 skips the item, and
+// an mbarrier parity wait is only sound for the phase right after the last one
+// its waiter saw, so S_FREE_0 must not advance on pages thread 1 does not follow.
 // Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
 // the kernel records a status word, every role stops, and TMEM is freed
 // before exit.
@@ -159,8 +163,9 @@ enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
   B_S_FULL,                  // 2: S = Q_w K^T computed into the S buffer
-  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (4 warp arrivals + the watcher)
-  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (4 warp arrivals + the watcher)
+  B_S_FREE = B_S_FULL + 2,   // 3: softmax w has loaded S (4 warp arrivals + the watcher);
+                             //    index 2 for the S tiles of single-tile items
+  B_P_FULL = B_S_FREE + 3,   // 2: P_w written (4 warp arrivals + the watcher)
   B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
   B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
@@ -260,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
     }
+    mbar_init(bar(B_S_FREE + 2), 5);  // softmax 0's 4 warps + the watcher, single-tile items
     for (int k = 0; k < kItemSlots; ++k) {
       mbar_init(bar(B_ITEM_FULL + k), 1);
       mbar_init(bar(B_ITEM_EMPTY + k), 3 + 8);  // MMA threads, watcher, one lane per softmax warp
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // been loaded (its S_FREE phase complete), both S MMAs are done with
       // K(t) and the watcher gives that slot back (both expected arrivals).
       if (lane == 0) {
-        uint32_t g = 0, sf[2] = {0, 0}, pf[2] = {0, 0};
+        uint32_t g = 0, sf[3] = {0, 0, 0}, pf[2] = {0, 0};
         bool ok = true;
         auto landed = [&](uint32_t r) -> bool {
           return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, 0x12a);
@@ -385,14 +391,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
           if (w.id >= p.n_items) break;
           const int nq = w.two ? 2 : 1;
+          // S_FREE barrier of tile q's S: a single-tile item's have their own.
+          auto sfb = [nq](int q) { return nq == 2 ? q : 2; };
           for (int t = 0; ok && t < w.n_pages; ++t, ++g) {
             for (int q = 0; ok && q < nq; ++q) {
               // S_FREE_q(t): if it lets S_0(t+1) go, K(t+1) must be in.
               if (q == nq - 1 && t + 1 < w.n_pages && !landed(2 * g + 2)) { ok = false; break; }
-              ok = next_phase(B_S_FREE, q, sf[q]);
+              ok = next_phase(B_S_FREE, sfb(q), sf[sfb(q)]);
             }
             // Page t's last S was loaded once that S_FREE completes: K(t) goes back.
-            if (ok) ok = wait_bar(bar(B_S_FREE + nq - 1), (sf[nq - 1] - 1) & 1, ctl, 0x12d);
+            if (ok) ok = wait_bar(bar(B_S_FREE + sfb(nq - 1)), (sf[sfb(nq - 1)] - 1) & 1, ctl, 0x12d);
             if (ok) mbar_arrive_cnt(bar(BR::RING_EMPTY + (2 * g) % S), 2);
             if (!ok || !landed(2 * g + 1)) { ok = false; break; }
             for (int q = 0; ok && q < nq; ++q) ok = next_phase(B_P_FULL, q, pf[q]);
@@ -410,9 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const int mw = warp == 1 ? 0 : 1;  // the query tile this thread issues for
         // g: pages walked; pv: P.V MMAs issued (P_mw buffers consumed);
-        // sc[w]: S MMAs issued so far for tile w (by either thread); itw:
-        // items done by tile mw; s_last: tile whose S the buffer holds.
-        uint32_t g = 0, it = 0, pv = 0, sc[2] = {0, 0}, itw = 0;
+        // sc[b]: S MMAs issued so far (by either thread) whose load signals
+        // S_FREE_b; itw: items done by tile mw; s_last: that barrier for the
+        // S the buffer holds.
+        uint32_t g = 0, it = 0, pv = 0, sc[3] = {0, 0, 0}, itw = 0;
         int s_last = -1;
         bool ok = true;
         auto ring_wait = [&](uint32_t r, int code) -> bool {
@@ -427,14 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
         auto lo_k = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | (1u << 16); };
         auto lo_mn = [](uint32_t addr) { return ((addr & 0x3FFFFu) >> 4) | ((16384u >> 4) << 16); };
-        // An S of tile w (ours or the other thread's) takes the buffer.
+        // An S (ours or the other thread's) takes the buffer; w names the
+        // S_FREE barrier its load signals (2: tile 0 of a single-tile item).
         auto take_s = [&](int w) {
           ++sc[w];
           s_last = w;
         };
         // S = Q_mw K(t)^T into the S buffer, once the buffer's previous owner
         // has loaded it.
-        auto issue_s = [&](uint32_t t) -> bool {
+        auto issue_s = [&](uint32_t t, int own) -> bool {
           if (s_last >= 0 &&
               !wait_bar(bar(B_S_FREE + s_last), (sc[s_last] - 1) & 1, ctl, 0x119 + s_last))
             return false;
@@ -453,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           tc_commit(bar(B_S_FULL + mw));
-          take_s(mw);
+          take_s(own);
           return true;
         };
         // O_mw (+)= P_mw V(t), once softmax mw has written P_mw (and, for an
@@ -464,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!accumulate && itw > 0 &&
               !wait_bar(bar(B_O_EMPTY + mw), (itw - 1) & 1, ctl, 0x114 + mw))
             return false;
-          // P_FULL implies V(t) has landed: the softmax checked it first.
+          // P_FULL implies V(t) has landed: the watcher joins it only then.
           tc_fence_after();
           const uint32_t vaddr = slot_addr(2 * t + 1);
           mma_ts_k128<2048 / 16>(tmem + C::kColO + 128 * mw, tmem + C::kColP + 64 * mw,
@@ -474,8 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         // V(t) goes back to the producer by one commit behind each tile's P.V
-        // (two from thread 0 with a single tile); K(t) by the softmax that
-        // sees the page's last S done.
+        // (two from thread 0 with a single tile); K(t) by the watcher once the
+        // page's last S has been loaded.
         auto release_v = [&](uint32_t t, int nq) {
           tc_commit(bar(BR::RING_EMPTY + (2 * t + 1) % S));
           if (nq == 1) tc_commit(bar(BR::RING_EMPTY + (2 * t + 1) % S));
@@ -492,19 +502,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = w.n_pages;
           const int nq = w.two ? 2 : 1;
           const uint32_t qit = it++;
-          if (mw >= nq) {  // the item has no tile for this thread: follow the S chain only
-            for (int j = 0; j < n; ++j) take_s(0);
+          if (mw >= nq) {
+            // The item has no tile for this thread. Its S tiles signal S_FREE_2,
+            // which this thread never waits on: S_FREE_0 then advances only on
+            // pages this thread takes part in, so each of its waits there is
+            // for the phase right after the last one it saw (a parity wait
+            // cannot tell a phase from the one two later).
             g += n;
             continue;
           }
-          if (!wait_bar(bar(B_Q_FULL), qit & 1, ctl, 0x110)) { ok = false; break; }
+          // Thread 0 waits for both Q tiles; thread 1's first S waits for the
+          // S_FREE_0 of thread 0's, so it needs no Q_FULL wait of its own (it
+          // skips single-tile items, whose Q_FULL phases it would not see).
+          if (mw == 0 && !wait_bar(bar(B_Q_FULL), qit & 1, ctl, 0x110)) { ok = false; break; }
           for (int j = 0; j < n && ok; ++j, ++g) {
             if (mw == 1) take_s(0);  // thread 0's S_0(t) went first
             // K(t) has landed: for an item's first page this thread checks;
-            // later, the S_FREE it waits for implies it (thread 1's S follows
-            // S_0(t); the softmax that frees the buffer for S_0(t) checked K(t)).
+            // later, the S_FREE it waits for implies it (the watcher joins the
+            // S_FREE that lets S_0(t) go only once K(t) is in, and thread 1's
+            // S follows S_0(t)).
             if (mw == 0 && j == 0 && !ring_wait(2 * g, 0x111)) { ok = false; break; }
-            if (!issue_s(g)) { ok = false; break; }
+            if (!issue_s(g, nq == 2 ? mw : 2)) { ok = false; break; }
             if (mw == nq - 1 && j == n - 1) tc_commit(bar(B_Q_EMPTY));  // the item's last S
             if (mw == 0 && nq == 2) take_s(1);  // thread 1's S_1(t) follows
             if (j > 0) {
@@ -561,13 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The whole S row in one TMEM round trip; then the S buffer goes back
         // to the MMA thread for the other tile's (or the next page's) S.
         float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
-        tmem_wait_ld();
+        tmem_ld128_wait(tS, *reinterpret_cast<uint32_t(*)[128]>(sv));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + wq));
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + (w.two ? wq : 2)));
         if (valid < 128) {  // partial last page of an entry: drop the padding keys
 #pragma unroll
           for (int i = 0; i < 128; ++i) sv[i] = i < valid ? sv[i] : -INFINITY;
@@ -600,8 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
+            tmem_ld32_wait(tO + c * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(tO + c * 32, o);
@@ -678,8 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
+          tmem_ld32_wait(tO + c * 32, o);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             po[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
@@ -699,8 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
+        tmem_ld32_wait(tO + c * 32, o);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -710,6 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 4; ++v)
             orow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
+        __syncwarp();  // rows past the node skip the store: reconverge before the next tcgen05.ld
       }
       tc_fence_before();
       mbar_arrive(bar(B_O_EMPTY + wq));

@@ -245,8 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int c = 0; c < 8; ++c) {
           const int64_t col0 = (int64_t)nt * 256 + 32 * c;
           uint32_t v[32];
-          tmem_ld32(trow + 256 * acc + 32 * c, v);
-          tmem_wait_ld();
+          tmem_ld32_wait(trow + 256 * acc + 32 * c, v);
           float f[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
@@ -276,6 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                   pack_bf16x2(f[8 * j + 4], f[8 * j + 5]),
                                   pack_bf16x2(f[8 * j + 6], f[8 * j + 7]));
           }
+          __syncwarp();  // rows past M skip the store: reconverge before the next tcgen05.ld
         }
       } else {
         // QKV: the tile holds two head slices of 128 features each.
@@ -304,8 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t v[32];
-            tmem_ld32(trow + 256 * acc + 128 * h + 32 * c, v);
-            tmem_wait_ld();
+            tmem_ld32_wait(trow + 256 * acc + 128 * h + 32 * c, v);
             float f[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
@@ -332,6 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                             pack_bf16x2(f[8 * j + 4], f[8 * j + 5]),
                                             pack_bf16x2(f[8 * j + 6], f[8 * j + 7]));
             }
+            __syncwarp();  // Q rows past the node skip the store: reconverge before the next tcgen05.ld
           }
         }
       }

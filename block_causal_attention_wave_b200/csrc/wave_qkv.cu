@@ -171,8 +171,7 @@ __global__ void __launch_bounds__(kQkvThreads, 2) qkv_append_kernel(const __grid
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t v[32];
-      tmem_ld32(trow + 32 * c, v);
-      tmem_wait_ld();
+      tmem_ld32_wait(trow + 32 * c, v);
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
@@ -182,6 +181,7 @@ __global__ void __launch_bounds__(kQkvThreads, 2) qkv_append_kernel(const __grid
         for (int j = 0; j < 4; ++j)
           dst[c * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       }
+      __syncwarp();  // Q rows past the tokens skip the store: reconverge before the next tcgen05.ld
     }
   }
   tc_fence_before();
