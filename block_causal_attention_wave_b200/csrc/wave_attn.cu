@@ -40,10 +40,11 @@
 //            and gives each K slot back once the page's last S has been
 //            loaded (V slots go back by a commit behind each P.V), so neither
 //            the issuers nor the softmax do any ring work.
-// A node's last pair of query tiles may hold one tile. The S tiles of such a
-// single-tile item signal a third S_FREE barrier: thread 1 skips the item, and
-// an mbarrier parity wait is only sound for the phase right after the last one
-// its waiter saw, so S_FREE_0 must not advance on pages thread 1 does not follow.
+// A node's last pair of query tiles may hold one tile. Thread 1 skips such a
+// single-tile item while its S tiles advance S_FREE_0; an mbarrier parity wait
+// is only sound for the phase right after the last one its waiter saw, so
+// before its next S thread 1 waits (bounded) until the watcher's count of
+// pages whose last S has been loaded covers the skipped pages.
 // Every wait is bounded (by default 2 s; wave_kv_set_wait_limit); on timeout
 // the kernel records a status word, every role stops, and TMEM is freed
 // before exit.
@@ -163,9 +164,8 @@ enum : int {
   B_Q_FULL = 0,
   B_Q_EMPTY,
   B_S_FULL,                  // 2: S = Q_w K^T computed into the S buffer
-  B_S_FREE = B_S_FULL + 2,   // 3: softmax w has loaded S (4 warp arrivals + the watcher);
-                             //    index 2 for the S tiles of single-tile items
-  B_P_FULL = B_S_FREE + 3,   // 2: P_w written (4 warp arrivals + the watcher)
+  B_S_FREE = B_S_FULL + 2,   // 2: softmax w has loaded S (4 warp arrivals + the watcher)
+  B_P_FULL = B_S_FREE + 2,   // 2: P_w written (4 warp arrivals + the watcher)
   B_P_FREE = B_P_FULL + 2,   // 2: the P.V that read P_w is done
   B_O_FULL = B_P_FREE + 2,   // 2: last P.V of an item done
   B_O_EMPTY = B_O_FULL + 2,  // 2: epilogue has read O_w (128 arrivals)
@@ -182,7 +182,7 @@ struct Bars {
   static constexpr int kS = Cfg<D>::kSlots;
   static constexpr int RING_FULL = B_RING_FULL, RING_EMPTY = RING_FULL + kS,
                        COUNT = RING_EMPTY + kS;
-  static_assert(COUNT * 8 + 16 + 4 * kItemWords * kItemSlots <= 448, "barrier area");  // 448..: clock
+  static_assert(COUNT * 8 + 16 + 4 * kItemWords * kItemSlots + 4 <= 448, "barrier area");  // 448..: clock
 };
 
 // A work item: (node, head, pair of 128-row query tiles, key range). The
@@ -242,6 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * BR::COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 4);
   volatile int* item_q = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * BR::COUNT + 8);
+  // Pages whose last S has been loaded, as the watcher saw them (monotonic).
+  volatile uint32_t* s_done = reinterpret_cast<volatile uint32_t*>(
+      smem + C::kBarOff + 8 * BR::COUNT + 8 + 4 * kItemWords * kItemSlots);
   const Ctl ctl{abort_flag, p.status, p.wait_ns};
 
   const int warp = threadIdx.x >> 5;
@@ -265,7 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_O_FULL + w), 1);
       mbar_init(bar(B_O_EMPTY + w), 128);
     }
-    mbar_init(bar(B_S_FREE + 2), 5);  // softmax 0's 4 warps + the watcher, single-tile items
     for (int k = 0; k < kItemSlots; ++k) {
       mbar_init(bar(B_ITEM_FULL + k), 1);
       mbar_init(bar(B_ITEM_EMPTY + k), 3 + 8);  // MMA threads, watcher, one lane per softmax warp
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BR::RING_EMPTY + s), 2);  // K: one arrival of 2; V: a commit per tile
     }
     *abort_flag = 0;
+    *s_done = 0;
     fence_mbar_init();
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_kv);
@@ -372,9 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arrives on a barrier's next phase only after the previous one
       // completed, so it is never two phases ahead. Once page t's last S has
       // been loaded (its S_FREE phase complete), both S MMAs are done with
-      // K(t) and the watcher gives that slot back (both expected arrivals).
+      // K(t) and the watcher gives that slot back (both expected arrivals),
+      // and counts the page in s_done (read by MMA thread 1 after a skip).
       if (lane == 0) {
-        uint32_t g = 0, sf[3] = {0, 0, 0}, pf[2] = {0, 0};
+        uint32_t g = 0, sf[2] = {0, 0}, pf[2] = {0, 0};
         bool ok = true;
         auto landed = [&](uint32_t r) -> bool {
           return wait_bar(bar(BR::RING_FULL + r % S), (r / S) & 1, ctl, 0x12a);
@@ -391,16 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(B_ITEM_EMPTY + (k % kItemSlots)));
           if (w.id >= p.n_items) break;
           const int nq = w.two ? 2 : 1;
-          // S_FREE barrier of tile q's S: a single-tile item's have their own.
-          auto sfb = [nq](int q) { return nq == 2 ? q : 2; };
           for (int t = 0; ok && t < w.n_pages; ++t, ++g) {
             for (int q = 0; ok && q < nq; ++q) {
               // S_FREE_q(t): if it lets S_0(t+1) go, K(t+1) must be in.
               if (q == nq - 1 && t + 1 < w.n_pages && !landed(2 * g + 2)) { ok = false; break; }
-              ok = next_phase(B_S_FREE, sfb(q), sf[sfb(q)]);
+              ok = next_phase(B_S_FREE, q, sf[q]);
             }
             // Page t's last S was loaded once that S_FREE completes: K(t) goes back.
-            if (ok) ok = wait_bar(bar(B_S_FREE + sfb(nq - 1)), (sf[sfb(nq - 1)] - 1) & 1, ctl, 0x12d);
+            if (ok) ok = wait_bar(bar(B_S_FREE + nq - 1), (sf[nq - 1] - 1) & 1, ctl, 0x12d);
+            if (ok) *s_done = g + 1;
             if (ok) mbar_arrive_cnt(bar(BR::RING_EMPTY + (2 * g) % S), 2);
             if (!ok || !landed(2 * g + 1)) { ok = false; break; }
             for (int q = 0; ok && q < nq; ++q) ok = next_phase(B_P_FULL, q, pf[q]);
@@ -421,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sc[b]: S MMAs issued so far (by either thread) whose load signals
         // S_FREE_b; itw: items done by tile mw; s_last: that barrier for the
         // S the buffer holds.
-        uint32_t g = 0, it = 0, pv = 0, sc[3] = {0, 0, 0}, itw = 0;
+        uint32_t g = 0, it = 0, pv = 0, sc[2] = {0, 0}, itw = 0;
+        bool resync = false;  // thread 1 skipped an item since its last S
         int s_last = -1;
         bool ok = true;
         auto ring_wait = [&](uint32_t r, int code) -> bool {
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // S = Q_mw K(t)^T into the S buffer, once the buffer's previous owner
         // has loaded it.
-        auto issue_s = [&](uint32_t t, int own) -> bool {
+        auto issue_s = [&](uint32_t t) -> bool {
           if (s_last >= 0 &&
               !wait_bar(bar(B_S_FREE + s_last), (sc[s_last] - 1) & 1, ctl, 0x119 + s_last))
             return false;
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           tc_commit(bar(B_S_FULL + mw));
-          take_s(own);
+          take_s(mw);
           return true;
         };
         // O_mw (+)= P_mw V(t), once softmax mw has written P_mw (and, for an
@@ -503,18 +507,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nq = w.two ? 2 : 1;
           const uint32_t qit = it++;
           if (mw >= nq) {
-            // The item has no tile for this thread. Its S tiles signal S_FREE_2,
-            // which this thread never waits on: S_FREE_0 then advances only on
-            // pages this thread takes part in, so each of its waits there is
-            // for the phase right after the last one it saw (a parity wait
-            // cannot tell a phase from the one two later).
+            // The item has no tile for this thread: its S tiles advance
+            // S_FREE_0 without this thread's waits, so before its next S it
+            // lets the watcher's page count catch up (a parity wait is only
+            // sound for the phase right after the last one its waiter saw).
+            for (int j = 0; j < n; ++j) take_s(0);
             g += n;
+            resync = true;
             continue;
           }
           // Thread 0 waits for both Q tiles; thread 1's first S waits for the
           // S_FREE_0 of thread 0's, so it needs no Q_FULL wait of its own (it
           // skips single-tile items, whose Q_FULL phases it would not see).
           if (mw == 0 && !wait_bar(bar(B_Q_FULL), qit & 1, ctl, 0x110)) { ok = false; break; }
+          if (resync) {  // every S before this item's has been loaded
+            const uint64_t t0 = globaltimer_ns();
+            while (ok && *s_done < g) {
+              __nanosleep(64);
+              if (*abort_flag) ok = false;
+              else if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+                *abort_flag = 1;
+                atomicCAS(p.status, 0, 0x11c);
+                ok = false;
+              }
+            }
+            if (!ok) break;
+            resync = false;
+          }
           for (int j = 0; j < n && ok; ++j, ++g) {
             if (mw == 1) take_s(0);  // thread 0's S_0(t) went first
             // K(t) has landed: for an item's first page this thread checks;
@@ -522,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S_FREE that lets S_0(t) go only once K(t) is in, and thread 1's
             // S follows S_0(t)).
             if (mw == 0 && j == 0 && !ring_wait(2 * g, 0x111)) { ok = false; break; }
-            if (!issue_s(g, nq == 2 ? mw : 2)) { ok = false; break; }
+            if (!issue_s(g)) { ok = false; break; }
             if (mw == nq - 1 && j == n - 1) tc_commit(bar(B_Q_EMPTY));  // the item's last S
             if (mw == 0 && nq == 2) take_s(1);  // thread 1's S_1(t) follows
             if (j > 0) {
@@ -582,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld128_wait(tS, *reinterpret_cast<uint32_t(*)[128]>(sv));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + (w.two ? wq : 2)));
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + wq));
         if (valid < 128) {  // partial last page of an entry: drop the padding keys
 #pragma unroll
           for (int i = 0; i < 128; ++i) sv[i] = i < valid ? sv[i] : -INFINITY;
