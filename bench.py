@@ -92,15 +92,15 @@ def _kernel_source_hash():
     return h.hexdigest()
 
 
-def _measured_traffic():
+def _measured_traffic(workload):
     """DRAM bytes per attention launch from the committed ncu capture, if it was
-    taken on the current kernel source (else None)."""
+    taken on the current kernel source and on this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "round_attn_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("kernel_source_sha256") != _kernel_source_hash():
+    if rec.get("kernel_source_sha256") != _kernel_source_hash() or rec.get("workload_key") != workload:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -114,15 +114,15 @@ def _source_hash(names):
     return h.hexdigest()
 
 
-def _measured_append_traffic():
+def _measured_append_traffic(workload):
     """DRAM bytes of the batched append launch from the committed ncu record, if
-    it was taken on the current append source (else None)."""
+    it was taken on the current append source and on this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "kv_append_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("kernel_source_sha256") != _source_hash(["wave_device.cu"]):
+    if rec.get("kernel_source_sha256") != _source_hash(["wave_device.cu"]) or rec.get("workload_key") != workload:
         return None
     return {k: rec.get(k) for k in ("dram_read_bytes", "dram_write_bytes", "duration_ns")}
 
@@ -531,7 +531,7 @@ def run_gpu(args):
                         "previous step's compute (double-buffered device buffers)"},
         "roofline": {"bound": "tensor", "kernel": "round_attn_kernel<128>",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": _measured_traffic(),
+                     "frac": round(achieved / peak, 4), "traffic": _measured_traffic(spec.key),
                      "peak_source": f"{src} bf16_tflops (burst, cuBLAS 8192^3)",
                      "flops_per_launch": flops, "avg_launch_ms": round(attn_avg, 4),
                      "effective_sm_mhz": round(eff_mhz, 1) if eff_mhz else None,
@@ -545,7 +545,7 @@ def run_gpu(args):
                    "peak_gbs": peaks["hbm_gbs"],
                    "frac": round(append_bytes / (append_ms * 1e-3) / 1e9 /
                                  peaks["hbm_gbs"], 4),
-                   "ncu": _measured_append_traffic(),
+                   "ncu": _measured_append_traffic(spec.key),
                    "ncu_note": "DRAM bytes of one batched append launch (ncu): writes that are "
                                "still in L2 when the kernel ends reach DRAM later"},
         "gpu_launches": K * 2,
