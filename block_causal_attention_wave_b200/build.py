@@ -31,8 +31,11 @@ def sources():
     return sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cpp")))
 
 
-def build(verbose_ptxas: bool = False, out: str = LIB, defines=()) -> str:
-    """Compile every source into ``out``; ``defines`` are extra -D macros."""
+def build(verbose_ptxas: bool = False, out: str = LIB, defines=(), replace=None) -> str:
+    """Compile every source into ``out``; ``defines`` are extra -D macros;
+    ``replace`` maps a source's file name to another file compiled in its place
+    (a test build of one kernel; headers still come from ``csrc``)."""
+    replace = dict(replace or {})
     objdir = os.path.join(PKG, "_build", os.path.splitext(os.path.basename(out))[0])
     os.makedirs(objdir, exist_ok=True)
     common = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-Wall",
@@ -43,6 +46,7 @@ def build(verbose_ptxas: bool = False, out: str = LIB, defines=()) -> str:
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        src = replace.pop(os.path.basename(src), src)
         cmd = [nvcc()] + common + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
         if r.returncode != 0 or verbose_ptxas:
@@ -50,6 +54,8 @@ def build(verbose_ptxas: bool = False, out: str = LIB, defines=()) -> str:
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
         objs.append(obj)
+    if replace:
+        raise ValueError(f"no source named {sorted(replace)}")
     tmp = out + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
