@@ -22,7 +22,9 @@ reports:
 ``protocol="original"`` models the protocol before the single-tile fix: both
 MMA threads wait for Q_FULL, and the second one, after skipping a single-tile
 item, takes its next S_FREE_0 parity wait without first waiting for the
-watcher's page count.
+watcher's page count. ``protocol="lean-watcher"`` is the current protocol with
+the watcher joining each S_FREE / P_FULL phase without first waiting for the
+previous phase to complete (those waits are implied by its other waits).
 """
 from __future__ import annotations
 
@@ -216,7 +218,7 @@ def watcher(st: State):
     sf, pf = [0, 0], [0, 0]
 
     def next_phase(base, q, n):
-        if n[q] > 0:
+        if n[q] > 0 and st.protocol != "lean-watcher":
             yield wait(f"{base}{q}", n[q] - 1)
         st.bar(f"{base}{q}").arrive()
         n[q] += 1
@@ -288,7 +290,7 @@ def issuer(st: State, mw: int):
             for _ in range(n):
                 take_s(0)
             g += n
-            resync = st.protocol == "current"
+            resync = st.protocol != "original"
             continue
         if mw == 0 or st.protocol == "original":
             yield wait("Q_FULL", qit)

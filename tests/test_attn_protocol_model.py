@@ -6,7 +6,8 @@ with the kernel's counters, waits, arrivals and commits, and runs them under a
 seeded random interleaving against a model of mbarrier phases, an in-order
 tensor pipe and delayed copies. These tests run many interleavings:
 - the protocol as built finishes every random item mix, single-tile items
-  included, with no early parity pass, no stall and no data hazard;
+  included, with no early parity pass, no stall and no data hazard, and so
+  does a watcher that joins each phase without waiting for the previous one;
 - the protocol before the single-tile fix is caught: with single-tile items in
   the mix, runs end in data hazards (an S MMA reading a K slot that does not
   hold its page, a copy into a slot an MMA still has to read); with two-tile
@@ -39,6 +40,13 @@ def test_current_protocol_is_clean():
 def test_current_protocol_single_tile_heavy_and_long():
     assert not _violations("current", p_single=0.8), "single-tile heavy"
     assert not _violations("current", p_single=0.4, count=30, max_pages=7, seeds=60), "long"
+
+
+def test_watcher_previous_phase_waits_are_implied():
+    """Joining S_FREE / P_FULL without waiting for the previous phase stays clean:
+    the watcher's other waits already imply those phases are complete."""
+    bad = _violations("lean-watcher", p_single=0.4)
+    assert not bad, bad[:3]
 
 
 def test_original_protocol_is_caught_on_single_tile_items():
