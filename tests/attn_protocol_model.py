@@ -31,7 +31,7 @@ from __future__ import annotations
 import random
 from dataclasses import dataclass, field
 
-RING_SLOTS = 5
+RING_SLOTS = 5     # d = 128 (the d = 64 kernel has 10)
 ITEM_SLOTS = 2
 SOFTMAX_WARPS = 4  # per warpgroup
 
@@ -73,12 +73,13 @@ class State:
     items: list
     rng: random.Random
     protocol: str = "current"
+    slots: int = RING_SLOTS
     bars: dict = field(default_factory=dict)
     item_q: list = field(default_factory=lambda: [None] * ITEM_SLOTS)
     s_done: int = 0
     # data
-    ring: list = field(default_factory=lambda: [None] * RING_SLOTS)  # (kind, page, landed)
-    ring_readers: list = field(default_factory=lambda: [0] * RING_SLOTS)  # MMAs queued on a slot
+    ring: list = field(default_factory=list)          # per slot: (kind, page, landed)
+    ring_readers: list = field(default_factory=list)  # per slot: MMAs queued on it
     q_buf: object = None                  # (item id, landed)
     s_buf: object = None                  # (tile, page)
     s_loaded: set = field(default_factory=set)
@@ -94,7 +95,7 @@ class State:
         return self.bars[name]
 
 
-def make_bars():
+def make_bars(slots: int = RING_SLOTS):
     b = {}
     def add(name, count):
         b[name] = Bar(name, count)
@@ -110,7 +111,7 @@ def make_bars():
     for k in range(ITEM_SLOTS):
         add(f"ITEM_FULL{k}", 1)
         add(f"ITEM_EMPTY{k}", 3 + 2 * SOFTMAX_WARPS)
-    for s in range(RING_SLOTS):
+    for s in range(slots):
         add(f"RING_FULL{s}", 1)
         add(f"RING_EMPTY{s}", 2)
     return b
@@ -138,7 +139,7 @@ def execute(st: State, op):
         _, w, page, item = op
         if st.s_buf is not None and len(st.s_loaded) < SOFTMAX_WARPS:
             raise Violation(f"S_{w}({page}) overwrites S{st.s_buf} loaded by {len(st.s_loaded)} warps")
-        slot = (2 * page) % RING_SLOTS
+        slot = (2 * page) % st.slots
         if st.ring[slot] != ("K", page, True):
             raise Violation(f"S_{w}({page}) reads K slot {slot} holding {st.ring[slot]}")
         st.ring_readers[slot] -= 1
@@ -147,7 +148,7 @@ def execute(st: State, op):
         st.s_buf, st.s_loaded = (w, page), set()
     elif kind == "PV":
         _, w, page, acc = op
-        slot = (2 * page + 1) % RING_SLOTS
+        slot = (2 * page + 1) % st.slots
         if st.ring[slot] != ("V", page, True):
             raise Violation(f"PV_{w}({page}) reads V slot {slot} holding {st.ring[slot]}")
         st.ring_readers[slot] -= 1
@@ -190,9 +191,9 @@ def producer(st: State):
         it += 1
         for _ in range(w.n):
             for kind in ("K", "V"):
-                s = r % RING_SLOTS
-                if r >= RING_SLOTS:
-                    yield wait(f"RING_EMPTY{s}", r // RING_SLOTS - 1)
+                s = r % st.slots
+                if r >= st.slots:
+                    yield wait(f"RING_EMPTY{s}", r // st.slots - 1)
                 if st.ring_readers[s]:
                     raise Violation(f"copy into slot {s} with {st.ring_readers[s]} MMAs to read it")
                 page = r // 2
@@ -231,12 +232,12 @@ def watcher(st: State):
         for t in range(w.n):
             for q in range(nq):
                 if q == nq - 1 and t + 1 < w.n:
-                    yield wait(f"RING_FULL{(2 * g + 2) % RING_SLOTS}", (2 * g + 2) // RING_SLOTS)
+                    yield wait(f"RING_FULL{(2 * g + 2) % st.slots}", (2 * g + 2) // st.slots)
                 yield from next_phase("S_FREE", q, sf)
             yield wait(f"S_FREE{nq - 1}", sf[nq - 1] - 1)
             st.s_done = g + 1
-            st.bar(f"RING_EMPTY{(2 * g) % RING_SLOTS}").arrive(2)
-            yield wait(f"RING_FULL{(2 * g + 1) % RING_SLOTS}", (2 * g + 1) // RING_SLOTS)
+            st.bar(f"RING_EMPTY{(2 * g) % st.slots}").arrive(2)
+            yield wait(f"RING_FULL{(2 * g + 1) % st.slots}", (2 * g + 1) // st.slots)
             for q in range(nq):
                 yield from next_phase("P_FULL", q, pf)
             g += 1
@@ -257,7 +258,7 @@ def issuer(st: State, mw: int):
     def issue_s(t, item):
         if s_last >= 0:
             yield wait(f"S_FREE{s_last}", sc[s_last] - 1)
-        st.ring_readers[(2 * t) % RING_SLOTS] += 1
+        st.ring_readers[(2 * t) % st.slots] += 1
         mma(st, ("S", mw, t, item))
         commit(st, f"S_FULL{mw}")
         take_s(mw)
@@ -267,16 +268,16 @@ def issuer(st: State, mw: int):
         yield wait(f"P_FULL{mw}", pv)
         if not acc and itw > 0:
             yield wait(f"O_EMPTY{mw}", itw - 1)
-        st.ring_readers[(2 * t + 1) % RING_SLOTS] += 1
+        st.ring_readers[(2 * t + 1) % st.slots] += 1
         st.p_queued[mw] += 1
         mma(st, ("PV", mw, t, acc))
         commit(st, f"P_FREE{mw}")
         pv += 1
 
     def release_v(t, nq):
-        commit(st, f"RING_EMPTY{(2 * t + 1) % RING_SLOTS}")
+        commit(st, f"RING_EMPTY{(2 * t + 1) % st.slots}")
         if nq == 1:
-            commit(st, f"RING_EMPTY{(2 * t + 1) % RING_SLOTS}")
+            commit(st, f"RING_EMPTY{(2 * t + 1) % st.slots}")
     k = 0
     while True:
         w = yield from next_item(st, k)
@@ -301,7 +302,7 @@ def issuer(st: State, mw: int):
             if mw == 1:
                 take_s(0)
             if mw == 0 and j == 0:
-                yield wait(f"RING_FULL{(2 * g) % RING_SLOTS}", (2 * g) // RING_SLOTS)
+                yield wait(f"RING_FULL{(2 * g) % st.slots}", (2 * g) // st.slots)
             yield from issue_s(g, w.id)
             if mw == nq - 1 and j == n - 1:
                 commit(st, "Q_EMPTY")
@@ -362,12 +363,13 @@ def softmax_warp(st: State, wq: int, warp: int):
 # ---------------------------------------------------------------- scheduler
 
 def run(items, seed: int, protocol: str = "current", early_fatal: bool = True,
-        max_steps: int = 200000):
+        slots: int = RING_SLOTS, max_steps: int = 200000):
     """Interleave every role and event at random until all roles finish.
     Raises Violation on a stall or a data hazard, and on an early pass unless
     ``early_fatal`` is False (then early passes are listed in ``state.early``)."""
-    st = State(items=list(items), rng=random.Random(seed), protocol=protocol)
-    st.bars = make_bars()
+    st = State(items=list(items), rng=random.Random(seed), protocol=protocol, slots=slots)
+    st.ring, st.ring_readers = [None] * slots, [0] * slots
+    st.bars = make_bars(slots)
     roles = {"producer": producer(st), "issuer0": issuer(st, 0), "issuer1": issuer(st, 1),
              "watcher": watcher(st)}
     for wq in range(2):

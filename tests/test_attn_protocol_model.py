@@ -21,12 +21,13 @@ import attn_protocol_model as m
 SEEDS = 300
 
 
-def _violations(protocol, p_single, count=10, max_pages=4, early_fatal=True, seeds=SEEDS):
+def _violations(protocol, p_single, count=10, max_pages=4, early_fatal=True, seeds=SEEDS,
+                slots=m.RING_SLOTS):
     bad = []
     for seed in range(seeds):
         items = m.random_items(random.Random(seed), count, max_pages=max_pages, p_single=p_single)
         try:
-            m.run(items, seed, protocol=protocol, early_fatal=early_fatal)
+            m.run(items, seed, protocol=protocol, early_fatal=early_fatal, slots=slots)
         except m.Violation as e:
             bad.append((seed, str(e)))
     return bad
@@ -40,6 +41,11 @@ def test_current_protocol_is_clean():
 def test_current_protocol_single_tile_heavy_and_long():
     assert not _violations("current", p_single=0.8), "single-tile heavy"
     assert not _violations("current", p_single=0.4, count=30, max_pages=7, seeds=60), "long"
+
+
+def test_current_protocol_with_the_d64_ring():
+    """The d = 64 kernel streams K/V through 10 ring slots instead of 5."""
+    assert not _violations("current", p_single=0.4, max_pages=8, slots=10)
 
 
 def test_watcher_previous_phase_waits_are_implied():
