@@ -38,7 +38,9 @@ def test_held_single_tile_items(cuda_lib, tmp_path):
     assert text.count(ANCHOR) == 1, "the S-row load statement moved: update the anchor"
     held_src = tmp_path / "wave_attn.cu"
     held_src.write_text(text.replace(ANCHOR, HOLD + ANCHOR))
-    lib = build.build(out=str(tmp_path / "libwave_held.so"),
+    # Built in-tree (the package's git-ignored _build folder), like the library itself.
+    os.makedirs(os.path.join(build.PKG, "_build"), exist_ok=True)
+    lib = build.build(out=os.path.join(build.PKG, "_build", "libwave_held.so"),
                       replace={"wave_attn.cu": str(held_src)})
 
     out = tmp_path / "held.npy"
